@@ -1,0 +1,167 @@
+/*
+ * xlstm_mlstm.h -- C ABI of the B200 (sm_100a) mLSTM forward library.
+ *
+ * The operation (xLSTM page, obsidian-dorae222.pages.dev, section "mLSTM
+ * (matrix LSTM)", eq. 1-3, with the stabilizer of its "sLSTM" section):
+ *
+ *   m_t  = max(f~_t + m_{t-1}, i~_t)                       (log-space stabilizer)
+ *   f'_t = exp(f~_t + m_{t-1} - m_t),  i'_t = exp(i~_t - m_t)
+ *   C~_t = f'_t C~_{t-1} + i'_t v_t k_t^T                   (eq. 1, stabilized)
+ *   n~_t = f'_t n~_{t-1} + i'_t k_t                         (eq. 2, stabilized)
+ *   h~_t = C~_t q_t / max(|n~_t^T q_t|, exp(-m_t))          (eq. 3 without o_t)
+ *
+ * with q_t multiplied by desc->qk_scale first.  (C~, n~, m) is the stabilized
+ * state: the unstabilized state of eq. 1-2 is (e^m C~, e^m n~), and the readout
+ * above equals eq. 3's C q / max(|n^T q|, 1) exactly.  The output gate o_t of
+ * eq. 3 and the input projections of the page's listing are not part of this
+ * library: q, k, v, i~, f~ arrive already projected.
+ *
+ * Layouts (row-major, contiguous, device memory):
+ *   q, k    [B][H][T][d_qk]  qkv_dtype (bf16 or fp32)
+ *   v       [B][H][T][d_v]   qkv_dtype
+ *   i_pre   [B][H][T]        fp32   input-gate pre-activation i~
+ *   f_pre   [B][H][T]        fp32   forget-gate pre-activation f~ (log forget gate)
+ *   h_out   [B][H][T][d_v]   fp32   pre-gate output h~
+ *   C       [B][H][d_v][d_qk] fp32  row = value index, so C q is a row dot
+ *   n       [B][H][d_qk]     fp32
+ *   m       [B][H]           fp32
+ * The step call uses the same tensors with the T axis removed.
+ *
+ * Ownership and execution: every pointer is caller-owned device memory.  The
+ * library allocates nothing; scratch memory is the caller's workspace, sized
+ * by xlstm_mlstm_workspace_size().  Calls enqueue work on `stream` and return
+ * without synchronising; results are ready when the stream is.
+ *
+ * Errors: argument problems are reported synchronously, before anything is
+ * enqueued.  XLSTM_ERR_CUDA reports a launch failure (the CUDA error is left
+ * for cudaGetLastError).  Faults detected on the device (a bounded wait that
+ * gave up) are recorded in the workspace status block and read back with
+ * xlstm_mlstm_workspace_status().
+ */
+#ifndef XLSTM_MLSTM_H
+#define XLSTM_MLSTM_H
+
+#include <stddef.h>
+#include <stdint.h>
+#include <cuda_runtime_api.h>
+
+#if defined(__GNUC__)
+#define XLSTM_API __attribute__((visibility("default")))
+#else
+#define XLSTM_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    XLSTM_OK = 0,
+    XLSTM_ERR_INVALID_ARG = 1,  /* null/misaligned pointer, bad size, overlap   */
+    XLSTM_ERR_UNSUPPORTED = 2,  /* valid request this build has no kernel for   */
+    XLSTM_ERR_CUDA = 3,         /* a CUDA launch or enqueue failed              */
+    XLSTM_ERR_TIMEOUT = 4,      /* a bounded device-side wait gave up           */
+    XLSTM_ERR_WORKSPACE = 5     /* workspace missing or smaller than required   */
+} xlstm_status_t;
+
+typedef enum {
+    XLSTM_F32 = 0,
+    XLSTM_BF16 = 1
+} xlstm_dtype_t;
+
+typedef struct {
+    int32_t B, H;        /* batch, heads: >= 1                                   */
+    int32_t T;           /* sequence length: >= 0 (ignored by the step call)     */
+    int32_t d_qk, d_v;   /* head dims: multiples of 16 in [16, 512]              */
+    int32_t qkv_dtype;   /* xlstm_dtype_t of q, k, v                             */
+    float qk_scale;      /* multiplies q before use (1 = the page literally)     */
+    int32_t chunk;       /* chunk length L for the chunkwise call; 0 = 64        */
+} xlstm_mlstm_desc_t;
+
+/*
+ * Chunkwise-parallel forward over a whole sequence.
+ *
+ * Splits T into chunks of L tokens (the last one ragged).  Inside a chunk the
+ * unrolled recurrence is evaluated in parallel form:
+ *   F_t = sum_{r<=t} f~_r (cumulative log forget gate, reset every chunk),
+ *   m_t = F_t + max(m_0, max_{s<=t}(i~_s - F_s))   -- exactly the stabilizer,
+ *   h~_t = [e^{F_t+m_0-m_t} C~_0 q_t + sum_{s<=t} e^{F_t-F_s+i~_s-m_t}(q_t.k_s) v_s]
+ *          / max(|same with n~_0 and 1 in place of C~_0 and v_s|, e^{-m_t})
+ * and the state is carried from chunk to chunk in fp32.  bf16 inputs run on
+ * tcgen05 tensor cores (fp32 accumulation); fp32 inputs on fp32 CUDA cores.
+ *
+ *   C_in, n_in, m_in : initial state; all three NULL means zero state (m = 0),
+ *                      otherwise all three must be given.
+ *   h_out            : required when T > 0.
+ *   C_out, n_out, m_out : final state; each may be NULL (then not written).
+ *                      The canonical stabilizer m_T of the recurrence is
+ *                      written, with C~ and n~ in that gauge.
+ *   workspace        : device scratch of >= xlstm_mlstm_workspace_size(desc)
+ *                      bytes, 256-byte aligned; its first 16 bytes are the
+ *                      status block.  Calls sharing a workspace must not
+ *                      overlap on the device.
+ * Chunk lengths: 0 (= 64), 16, 32, 64; others return XLSTM_ERR_UNSUPPORTED.
+ * Outputs must not overlap inputs.  T = 0 copies the state through.
+ */
+XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise(
+    const xlstm_mlstm_desc_t *desc,
+    const void *q, const void *k, const void *v,
+    const float *i_pre, const float *f_pre,
+    const float *C_in, const float *n_in, const float *m_in,
+    float *h_out, float *C_out, float *n_out, float *m_out,
+    void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * Recurrent forward over a whole sequence: the recurrence above evaluated one
+ * token at a time with the state held on chip (O(1) state memory per head,
+ * O(T) time).  Same arguments and rules as xlstm_mlstm_fwd_chunkwise;
+ * desc->chunk is ignored; the workspace may be NULL (it needs none).
+ */
+XLSTM_API xlstm_status_t xlstm_mlstm_fwd_recurrent(
+    const xlstm_mlstm_desc_t *desc,
+    const void *q, const void *k, const void *v,
+    const float *i_pre, const float *f_pre,
+    const float *C_in, const float *n_in, const float *m_in,
+    float *h_out, float *C_out, float *n_out, float *m_out,
+    void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * One decode step (the page's forward_recurrent without projections and o_t):
+ *   q, k [B][H][d_qk], v [B][H][d_v], i_pre, f_pre [B][H];
+ *   C, n, m : state in (required);  h_out [B][H][d_v];
+ *   C_new, n_new, m_new : state out (required).  Each may equal its input
+ *   exactly (in-place update); any other overlap is rejected.
+ * desc->T and desc->chunk are ignored.  Memory-bound: C is read and written
+ * once with 128-bit coalesced accesses.
+ */
+XLSTM_API xlstm_status_t xlstm_mlstm_step(
+    const xlstm_mlstm_desc_t *desc,
+    const void *q, const void *k, const void *v,
+    const float *i_pre, const float *f_pre,
+    const float *C, const float *n, const float *m,
+    float *h_out, float *C_new, float *n_new, float *m_new,
+    cudaStream_t stream);
+
+/* Workspace bytes xlstm_mlstm_fwd_chunkwise needs for desc (>= 256), or 0 for
+ * a NULL desc. */
+XLSTM_API size_t xlstm_mlstm_workspace_size(const xlstm_mlstm_desc_t *desc);
+
+/*
+ * Reads the workspace status block written by the device: waits for `stream`,
+ * returns XLSTM_OK or the recorded device error (e.g. XLSTM_ERR_TIMEOUT), and
+ * stores the code of the wait that gave up in *where (may be NULL).
+ * Each chunkwise call clears the block before its kernels run.
+ */
+XLSTM_API xlstm_status_t xlstm_mlstm_workspace_status(const void *workspace, int32_t *where,
+                                            cudaStream_t stream);
+
+/* Human-readable name of a status code (static storage). */
+XLSTM_API const char *xlstm_status_string(xlstm_status_t status);
+
+/* Library version string (static storage). */
+XLSTM_API const char *xlstm_mlstm_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* XLSTM_MLSTM_H */

@@ -1,0 +1,105 @@
+"""Host-side checks of the C-ABI library (no GPU needed, no kernel launched).
+
+The library must load, export every entry point that include/*.h declares,
+and reject bad arguments synchronously, before touching the device.  Only
+argument checks that return before any CUDA call are exercised here.
+"""
+import glob
+import os
+import re
+
+import pytest
+
+from xlstm_mlstm_matrix_b200 import capi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    names = set()
+    for path in glob.glob(os.path.join(ROOT, "include", "*.h")):
+        text = open(path).read()
+        names.update(re.findall(r"XLSTM_API\s+[\w\s\*]*?\b(xlstm_\w+)\s*\(", text))
+    return sorted(names)
+
+
+@pytest.fixture(scope="module")
+def lib():
+    if not os.path.exists(capi.LIB_PATH):
+        from xlstm_mlstm_matrix_b200 import build
+        build.build()
+    return capi.load()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    names = declared_symbols()
+    assert len(names) >= 7, names
+    for n in names:
+        assert hasattr(lib, n), f"{n} declared in include/ but not exported"
+    assert set(capi.EXPORTED) <= set(names)
+
+
+def test_version_and_status_strings(lib):
+    assert "sm_100a" in capi.xlstm_mlstm_version()
+    assert capi.xlstm_status_string(capi.XLSTM_OK) == "ok"
+    assert "timed out" in capi.xlstm_status_string(capi.XLSTM_ERR_TIMEOUT)
+
+
+def test_workspace_size(lib):
+    d = capi.make_desc(8, 8, 4096, 256, 512)
+    assert capi.xlstm_mlstm_workspace_size(d) >= 256
+
+
+FAKE = dict(q=0x10000, k=0x20000, v=0x30000, i=0x40000, f=0x50000, h=0x60000, ws=0x100000)
+
+
+def call(desc, **over):
+    a = dict(FAKE, **over)
+    return capi.xlstm_mlstm_fwd_chunkwise(desc, a["q"], a["k"], a["v"], a["i"], a["f"],
+                                          a.get("C0"), a.get("n0"), a.get("m0"), a["h"],
+                                          a.get("C1"), a.get("n1"), a.get("m1"), a["ws"],
+                                          a.get("wsb", 256))
+
+
+@pytest.mark.parametrize("field,value", [("B", 0), ("H", -1), ("T", -1), ("d_qk", 8), ("d_qk", 520),
+                                         ("d_v", 24), ("d_v", 0), ("qkv_dtype", 7)])
+def test_bad_dims_rejected(lib, field, value):
+    d = capi.make_desc(1, 1, 4, 32, 32)
+    setattr(d, field, value)
+    assert call(d) == capi.XLSTM_ERR_INVALID_ARG
+
+
+def test_null_and_misaligned_pointers_rejected(lib):
+    d = capi.make_desc(1, 1, 4, 32, 32)
+    assert call(d, q=None) == capi.XLSTM_ERR_INVALID_ARG
+    assert call(d, h=None) == capi.XLSTM_ERR_INVALID_ARG
+    assert call(d, k=FAKE["k"] + 4) == capi.XLSTM_ERR_INVALID_ARG
+    assert call(d, ws=FAKE["ws"] + 16) == capi.XLSTM_ERR_INVALID_ARG
+    # partial state: all three or none
+    assert call(d, C0=0x70000) == capi.XLSTM_ERR_INVALID_ARG
+
+
+def test_overlaps_rejected(lib):
+    d = capi.make_desc(1, 1, 4, 32, 32)
+    assert call(d, h=FAKE["q"]) == capi.XLSTM_ERR_INVALID_ARG          # out over an input
+    assert call(d, C1=FAKE["h"] + 64) == capi.XLSTM_ERR_INVALID_ARG    # two outputs overlap
+
+
+def test_workspace_and_chunk_rules(lib):
+    d = capi.make_desc(1, 1, 4, 32, 32)
+    assert call(d, ws=None) == capi.XLSTM_ERR_WORKSPACE
+    assert call(d, wsb=8) == capi.XLSTM_ERR_WORKSPACE
+    d.chunk = 48
+    assert call(d) == capi.XLSTM_ERR_UNSUPPORTED
+
+
+def test_step_rejects_partial_in_place(lib):
+    d = capi.make_desc(2, 2, 1, 32, 32)
+    C, n, m = 0x70000, 0x80000, 0x90000
+    # C_new overlapping C without being identical
+    st = capi.xlstm_mlstm_step(d, FAKE["q"], FAKE["k"], FAKE["v"], FAKE["i"], FAKE["f"],
+                               C, n, m, FAKE["h"], C + 256, 0xA0000, 0xB0000)
+    assert st == capi.XLSTM_ERR_INVALID_ARG
+    st = capi.xlstm_mlstm_step(d, FAKE["q"], FAKE["k"], FAKE["v"], FAKE["i"], FAKE["f"],
+                               C, n, m, None, C, n, m)
+    assert st == capi.XLSTM_ERR_INVALID_ARG

@@ -1,0 +1,203 @@
+"""GPU parity: the three C-ABI calls against the float64 oracle (needs a B200).
+
+Small shapes run the oracle on every head; the full-size workloads run the GPU
+on the whole input, in the launch configuration the benchmark times, and the
+oracle on sampled heads (each head is an independent recurrence).
+Tolerances (per-row normalised relative error): fp32 inputs 1e-4; bf16 inputs
+2e-2 max and 4e-3 mean; m within 1e-4 max(1, |m|); states compared after
+fixing the gauge (C e^{m_gpu - m_ref}).
+"""
+import numpy as np
+import pytest
+import torch
+
+from gpu_helpers import compare, gpu_sequence, oracle_sequence, select_heads, to_dev
+import oracle
+from xlstm_mlstm_matrix_b200 import capi, inputs
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    assert torch.cuda.is_available(), "GPU tests need a CUDA device"
+    capi.load()
+
+
+SMALL = [  # B, H, T, dqk, dv
+    (1, 2, 1, 16, 16),
+    (2, 2, 17, 32, 48),
+    (1, 3, 100, 64, 64),
+    (2, 1, 130, 128, 32),
+    (1, 1, 64, 16, 128),
+    (1, 2, 200, 256, 64),
+]
+
+
+def small_inputs(B, H, T, dqk, dv, dtype, state, seed=7, gate="std", mean_i=0.0, std_i=1.5):
+    w = inputs.WORKLOADS["tiny_fp32"].replace(
+        B=B, H=H, T=T, d_qk=dqk, d_v=dv, dtype=dtype, gate=gate, mean_i=mean_i, std_i=std_i,
+        state="normal_m_uniform" if state else "zero", seed=seed)
+    return inputs.make_sequence(w)
+
+
+@pytest.mark.parametrize("kind", ["chunkwise", "recurrent"])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+@pytest.mark.parametrize("shape", SMALL, ids=lambda s: "x".join(map(str, s)))
+@pytest.mark.parametrize("state", [False, True])
+def test_small_shapes(kind, dtype, shape, state):
+    inp = small_inputs(*shape, dtype, state, seed=sum(shape))
+    for scale in (1.0, shape[3] ** -0.5):
+        got = gpu_sequence(inp, kind, qk_scale=scale)
+        ref = oracle_sequence(inp, qk_scale=scale)
+        compare(got, ref, dtype, f"{kind} {dtype} {shape} state={state} scale={scale:.3f}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_chunk_size_invariance(dtype):
+    inp = small_inputs(2, 2, 203, 64, 64, dtype, True, seed=3)
+    ref = oracle_sequence(inp)
+    outs = {}
+    for L in (16, 32, 64):
+        outs[L] = gpu_sequence(inp, "chunkwise", chunk=L)
+        compare(outs[L], ref, dtype, f"L={L}")
+    tol = 1e-4 if dtype == "f32" else 2e-2
+    for L in (16, 32):
+        mx, _ = inputs.relative_errors(outs[L][0], outs[64][0])
+        assert mx <= tol, f"chunk {L} vs 64: {mx:.2e}"
+
+
+@pytest.mark.parametrize("gate,mean_i,std_i", [("mixed", 0.0, 1.0), ("std", 4.0, 6.0)])
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_stabilizer_stress(gate, mean_i, std_i, dtype):
+    """Positive log-forget gates (exp(f~) > 1) and large input-gate jumps."""
+    inp = small_inputs(2, 2, 300, 64, 64, dtype, True, seed=11, gate=gate, mean_i=mean_i, std_i=std_i)
+    ref = oracle_sequence(inp)
+    for kind in ("chunkwise", "recurrent"):
+        compare(gpu_sequence(inp, kind), ref, dtype, f"{kind} {gate}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_reset_gates(dtype):
+    """f~ = -1e4 at every token: each token forgets everything before it."""
+    inp = small_inputs(1, 2, 150, 64, 64, dtype, True, seed=5)
+    inp["f_pre"] = np.full_like(inp["f_pre"], -1.0e4)
+    ref = oracle_sequence(inp)
+    for kind in ("chunkwise", "recurrent"):
+        compare(gpu_sequence(inp, kind), ref, dtype, f"{kind} reset")
+
+
+def test_empty_sequence_passes_state_through():
+    inp = small_inputs(2, 2, 0, 32, 32, "bf16", True)
+    for kind in ("chunkwise", "recurrent"):
+        h, C, n, m = gpu_sequence(inp, kind)
+        assert h.shape == (2, 2, 0, 32)
+        np.testing.assert_array_equal(C, inp["C0"])
+        np.testing.assert_array_equal(n, inp["n0"])
+        np.testing.assert_array_equal(m, inp["m0"])
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_composition_across_calls(dtype):
+    """run(T1+T2) == run(T2, state=run(T1).state), mixing call types."""
+    inp = small_inputs(2, 2, 150, 64, 32, dtype, True, seed=9)
+    ref = oracle_sequence(inp)
+    s = 70
+    first = {k: (v[:, :, :s] if k in ("q", "k", "v", "i_pre", "f_pre") else v) for k, v in inp.items()}
+    second = {k: (v[:, :, s:] if k in ("q", "k", "v", "i_pre", "f_pre") else v) for k, v in inp.items()}
+    for k1, k2 in (("chunkwise", "chunkwise"), ("chunkwise", "recurrent"), ("recurrent", "chunkwise")):
+        h1, C1, n1, m1 = gpu_sequence(first, k1)
+        st = tuple(torch.from_numpy(x).cuda() for x in (C1, n1, m1))
+        h2, C2, n2, m2 = gpu_sequence(second, k2, state=st)
+        compare((np.concatenate([h1, h2], 2), C2, n2, m2), ref, dtype, f"{k1}->{k2}")
+
+
+@pytest.mark.parametrize("dtype", ["f32", "bf16"])
+def test_step_matches_oracle_and_recurrent(dtype):
+    B, H, T, dqk, dv = 3, 2, 40, 64, 96
+    inp = small_inputs(B, H, T, dqk, dv, dtype, True, seed=21)
+    ref = oracle_sequence(inp)
+    C = to_dev(inp["C0"], "f32"); n = to_dev(inp["n0"], "f32"); m = to_dev(inp["m0"], "f32")
+    hs = []
+    for t in range(T):
+        q, k, v = (to_dev(np.ascontiguousarray(inp[x][:, :, t]), dtype) for x in ("q", "k", "v"))
+        ig, fg = (to_dev(np.ascontiguousarray(inp[x][:, :, t]), "f32") for x in ("i_pre", "f_pre"))
+        h, (C, n, m) = capi.step(q, k, v, ig, fg, (C, n, m), qk_scale=inp["qk_scale"], inplace=(t % 2 == 0))
+        hs.append(h.cpu().numpy())
+    got = (np.stack(hs, 2), C.cpu().numpy(), n.cpu().numpy(), m.cpu().numpy())
+    compare(got, ref, dtype, "step x T")
+    compare(got, gpu_sequence(inp, "recurrent"), dtype, "step x T vs recurrent")
+
+
+def test_invalid_arguments_rejected():
+    d = capi.make_desc(1, 1, 8, 32, 32, capi.XLSTM_BF16, 1.0, 0)
+    q = torch.zeros(1, 1, 8, 32, device="cuda", dtype=torch.bfloat16)
+    g = torch.zeros(1, 1, 8, device="cuda")
+    h = torch.empty(1, 1, 8, 32, device="cuda")
+    ws = torch.zeros(256, device="cuda", dtype=torch.uint8)
+    f = capi.xlstm_mlstm_fwd_chunkwise
+    assert f(d, q, q, q, g, g, None, None, None, h, None, None, None, ws, 256) == capi.XLSTM_OK
+    # output aliasing an input
+    assert f(d, q, q, q, g, g, None, None, None, q, None, None, None, ws, 256) == capi.XLSTM_ERR_INVALID_ARG
+    # workspace missing / too small
+    assert f(d, q, q, q, g, g, None, None, None, h, None, None, None, None, 0) == capi.XLSTM_ERR_WORKSPACE
+    assert f(d, q, q, q, g, g, None, None, None, h, None, None, None, ws, 16) == capi.XLSTM_ERR_WORKSPACE
+    # misaligned pointer
+    assert f(d, q.data_ptr() + 2, q, q, g, g, None, None, None, h, None, None, None, ws, 256) == capi.XLSTM_ERR_INVALID_ARG
+    # unsupported chunk
+    d.chunk = 48
+    assert f(d, q, q, q, g, g, None, None, None, h, None, None, None, ws, 256) == capi.XLSTM_ERR_UNSUPPORTED
+    torch.cuda.synchronize()
+    assert capi.xlstm_mlstm_workspace_status(ws)[0] == capi.XLSTM_OK
+
+
+# ---- full-size workloads, sampled heads ------------------------------------------
+_cache = {}
+
+
+def full_inputs(name):
+    if name not in _cache:
+        _cache.clear()
+        _cache[name] = inputs.make_sequence(inputs.WORKLOADS[name])
+    return _cache[name]
+
+
+def test_tiny_fp32_full():
+    inp = full_inputs("tiny_fp32")
+    ref = oracle_sequence(inp)
+    for kind in ("chunkwise", "recurrent"):
+        compare(gpu_sequence(inp, kind), ref, "f32", f"tiny_fp32 {kind}")
+
+
+@pytest.mark.parametrize("name,heads", [("layer_7b", [0, 37, 63]), ("long_context", [2, 7]),
+                                        ("many_short", [0, 511, 1023])])
+@pytest.mark.parametrize("kind", ["chunkwise", "recurrent"])
+def test_full_size_sampled_heads(name, heads, kind):
+    inp = full_inputs(name)
+    got = gpu_sequence(inp, kind)
+    ref = oracle_sequence(inp, heads=heads)
+    got = tuple(select_heads(x, heads) for x in got)
+    compare(got, ref, inp["workload"].dtype, f"{name} {kind} heads {heads}")
+    assert np.all(np.isfinite(got[0]))
+
+
+def test_decode_256_steps_sampled_heads():
+    w = inputs.WORKLOADS["decode"]
+    rng, C0, n0, m0 = inputs.decode_state(w)
+    heads = [0, 300, 1023]
+    C, n, m = to_dev(C0, "f32"), to_dev(n0, "f32"), to_dev(m0, "f32")
+    scale = w.d_qk ** -0.5
+    hs, steps = [], []
+    for st in inputs.decode_steps(w, rng):
+        q, k, v = (to_dev(st[x], w.dtype) for x in ("q", "k", "v"))
+        ig, fg = to_dev(st["i_pre"], "f32"), to_dev(st["f_pre"], "f32")
+        h, (C, n, m) = capi.step(q, k, v, ig, fg, (C, n, m), qk_scale=scale, inplace=True)
+        hs.append(select_heads(h.cpu().numpy(), heads)[0])
+        steps.append({x: select_heads(st[x], heads)[0] for x in st})
+    seq = {x: np.stack([s[x] for s in steps], 1)[None] for x in steps[0]}
+    ref = oracle.forward(seq["q"], seq["k"], seq["v"], seq["i_pre"], seq["f_pre"],
+                         select_heads(C0, heads), select_heads(n0, heads), select_heads(m0, heads),
+                         qk_scale=scale)
+    got = (np.stack(hs, 1)[None], select_heads(C.cpu().numpy(), heads),
+           select_heads(n.cpu().numpy(), heads), select_heads(m.cpu().numpy(), heads))
+    compare(got, ref, w.dtype, "decode 256 steps")

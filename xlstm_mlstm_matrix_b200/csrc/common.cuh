@@ -1,0 +1,52 @@
+// Internal declarations shared by the kernels of the mLSTM library (sm_100a).
+#pragma once
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+
+#include "../../include/xlstm_mlstm.h"
+
+namespace xlstm {
+
+// Everything one forward launch needs, already validated by the C ABI layer.
+struct FwdArgs {
+    int B, H, T, dqk, dv;
+    int dtype;          // xlstm_dtype_t
+    float scale;        // qk_scale
+    int chunk;          // L (chunkwise only)
+    const void *q, *k, *v;
+    const float *ig, *fg;
+    const float *C0, *n0, *m0;   // all null = zero state
+    float *h, *C1, *n1, *m1;     // state outs may be null
+    int32_t *status;             // device status block (4 x int32), may be null
+};
+
+// Device status block layout (first 16 bytes of the workspace).
+enum : int32_t { kStatusCode = 0, kStatusWhere = 1 };
+
+cudaError_t launch_step(const FwdArgs &a, cudaStream_t s);
+cudaError_t launch_recurrent(const FwdArgs &a, cudaStream_t s);
+cudaError_t launch_chunkwise_simt(const FwdArgs &a, cudaStream_t s);
+bool chunkwise_tc_supported(const FwdArgs &a);
+cudaError_t launch_chunkwise_tc(const FwdArgs &a, cudaStream_t s);
+
+// ---- small device helpers ------------------------------------------------
+__device__ __forceinline__ float to_f32(float x) { return x; }
+__device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+__device__ __forceinline__ float warp_sum(float x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
+
+// Stabilized gates of one step: m' = max(f~ + m, i~), f' = e^{f~+m-m'}, i' = e^{i~-m'}.
+__device__ __forceinline__ void stabilized_gates(float fg, float ig, float m, float &m_new,
+                                                 float &fp, float &ip) {
+    const float a = fg + m;
+    m_new = (a > ig) ? a : ig;
+    fp = expf(a - m_new);
+    ip = expf(ig - m_new);
+}
+
+}  // namespace xlstm
