@@ -53,14 +53,66 @@ def select_heads(x, heads):
     return x.reshape((B * H,) + x.shape[2:])[heads][None]
 
 
-def compare(got, ref, dtype: str, what: str = "", check_state=True):
-    """got/ref: (h, C, n, m).  Raises AssertionError with the error figures."""
+def condition_numbers(inp, qk_scale=None, heads=None):
+    """Per-token condition numbers of the readout, in float64:
+      kappa_den_t = sum_j |n~_tj q_tj| / max(|sum_j n~_tj q_tj|, e^{-m_t})
+      kappa_num_t = max_r sum_j |C~_t,rj q_tj| / max_r |sum_j C~_t,rj q_tj|
+    A row of h~ is a dot product divided by a dot product; an fp32 evaluation
+    of either in any order carries a relative error of order
+    (kappa_den + kappa_num) * 2^-24 on that row, so where they cancel no fp32
+    kernel meets 1e-4.  These set tolerances only; nothing is compared with them."""
+    q, k, v, ig, fg = (inp[x].astype(np.float64) for x in ("q", "k", "v", "i_pre", "f_pre"))
+    C0, n0, m0 = inp.get("C0"), inp.get("n0"), inp.get("m0")
+    if heads is not None:
+        q, k, v, ig, fg = (select_heads(x, heads) for x in (q, k, v, ig, fg))
+        C0, n0, m0 = (None if x is None else select_heads(x, heads) for x in (C0, n0, m0))
+    scale = inp["qk_scale"] if qk_scale is None else qk_scale
+    B, H, T, dqk = q.shape
+    dv = v.shape[-1]
+    C = np.zeros((B, H, dv, dqk)) if C0 is None else C0.astype(np.float64).copy()
+    n = np.zeros((B, H, dqk)) if n0 is None else n0.astype(np.float64).copy()
+    m = np.zeros((B, H)) if m0 is None else m0.astype(np.float64).copy()
+    kd = np.ones((B, H, T))
+    kn = np.ones((B, H, T))
+    for t in range(T):
+        mn = np.maximum(fg[:, :, t] + m, ig[:, :, t])
+        fp = np.exp(fg[:, :, t] + m - mn)
+        ip = np.exp(ig[:, :, t] - mn)
+        C = fp[..., None, None] * C + ip[..., None, None] * v[:, :, t, :, None] * k[:, :, t, None, :]
+        n = fp[..., None] * n + ip[..., None] * k[:, :, t]
+        qs = scale * q[:, :, t]
+        prod = n * qs
+        kd[:, :, t] = np.abs(prod).sum(-1) / np.maximum(np.abs(prod.sum(-1)), np.exp(-mn))
+        mag = np.einsum("bhrc,bhc->bhr", np.abs(C), np.abs(qs)).max(-1)
+        val = np.abs(np.einsum("bhrc,bhc->bhr", C, qs)).max(-1)
+        kn[:, :, t] = mag / np.where(val > 0, val, 1.0)
+        m = mn
+    return kd, kn
+
+
+def fp32_row_tolerance(inp, qk_scale=None, heads=None, base=1e-4):
+    """max(base, 32 * 2^-24 * (kappa_den + kappa_num)) per (b, h, t) row."""
+    kd, kn = condition_numbers(inp, qk_scale, heads)
+    return np.maximum(base, 32.0 * 2.0 ** -24 * (kd + kn))
+
+
+def compare(got, ref, dtype: str, what: str = "", check_state=True, row_tol=None):
+    """got/ref: (h, C, n, m).  Raises AssertionError with the error figures.
+    row_tol: per-(b, h, t) tolerance for fp32 inputs (fp32_row_tolerance);
+    without it every row must meet 1e-4."""
     tol = TOL[dtype]
     h, C, n, m = got
     hr, Cr, nr, mr = ref
     mx, mean = inputs.relative_errors(h, hr)
     msgs = [f"h max {mx:.2e} mean {mean:.2e}"]
-    ok = mx <= tol["max"] and mean <= tol["mean"]
+    if row_tol is not None and dtype == "f32" and h.size:
+        scale = np.max(np.abs(hr), axis=-1, keepdims=True)
+        err = np.abs(h.astype(np.float64) - hr) / np.where(scale > 0, scale, 1.0)
+        worst = float(np.max(err / row_tol[..., None]))
+        msgs.append(f"h max/row-tol {worst:.2f} (row-tol max {float(np.max(row_tol)):.1e})")
+        ok = worst <= 1.0 and mean <= tol["mean"]
+    else:
+        ok = mx <= tol["max"] and mean <= tol["mean"]
     if check_state:
         # gauge-fixed state: C_gpu e^{m_gpu - m_ref} against C_ref
         g = np.exp(m.astype(np.float64) - mr)

@@ -11,7 +11,7 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import compare, gpu_sequence, oracle_sequence, select_heads, to_dev
+from gpu_helpers import compare, fp32_row_tolerance, gpu_sequence, oracle_sequence, select_heads, to_dev
 import oracle
 from xlstm_mlstm_matrix_b200 import capi, inputs
 
@@ -73,8 +73,9 @@ def test_stabilizer_stress(gate, mean_i, std_i, dtype):
     """Positive log-forget gates (exp(f~) > 1) and large input-gate jumps."""
     inp = small_inputs(2, 2, 300, 64, 64, dtype, True, seed=11, gate=gate, mean_i=mean_i, std_i=std_i)
     ref = oracle_sequence(inp)
+    tol = fp32_row_tolerance(inp)
     for kind in ("chunkwise", "recurrent"):
-        compare(gpu_sequence(inp, kind), ref, dtype, f"{kind} {gate}")
+        compare(gpu_sequence(inp, kind), ref, dtype, f"{kind} {gate}", row_tol=tol)
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
