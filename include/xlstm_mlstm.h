@@ -161,6 +161,24 @@ XLSTM_API const char *xlstm_status_string(xlstm_status_t status);
 /* Library version string (static storage). */
 XLSTM_API const char *xlstm_mlstm_version(void);
 
+/*
+ * Which kernel xlstm_mlstm_fwd_chunkwise runs for desc: "tcgen05" (bf16
+ * inputs, chunk 64, d_qk in {64, 128, 256}, d_v a multiple of 128), "simt"
+ * (fp32 CUDA-core kernel: fp32 inputs and every other supported shape),
+ * "copy" (T = 0) or "none" (invalid or unsupported desc).  Static storage.
+ */
+XLSTM_API const char *xlstm_mlstm_chunkwise_kernel(const xlstm_mlstm_desc_t *desc);
+
+/*
+ * Testing hook for the device-side bounded waits.  When enable != 0, the next
+ * tcgen05 chunkwise launch withholds one internal hand-off, so that the waits
+ * depending on it run out after their 1 s limit: the kernel then records
+ * XLSTM_ERR_TIMEOUT in the workspace status block, drains its in-flight copies
+ * and tensor-core work, frees its tensor memory and returns (its outputs are
+ * not valid).  The flag is consumed by that one launch.  No other effect.
+ */
+XLSTM_API void xlstm_mlstm_test_timeout_next(int32_t enable);
+
 #ifdef __cplusplus
 }
 #endif

@@ -74,6 +74,7 @@ def condition_numbers(inp, qk_scale=None, heads=None):
     m = np.zeros((B, H)) if m0 is None else m0.astype(np.float64).copy()
     kd = np.ones((B, H, T))
     kn = np.ones((B, H, T))
+    mabs = np.zeros((B, H, T))
     for t in range(T):
         mn = np.maximum(fg[:, :, t] + m, ig[:, :, t])
         fp = np.exp(fg[:, :, t] + m - mn)
@@ -86,14 +87,19 @@ def condition_numbers(inp, qk_scale=None, heads=None):
         mag = np.einsum("bhrc,bhc->bhr", np.abs(C), np.abs(qs)).max(-1)
         val = np.abs(np.einsum("bhrc,bhc->bhr", C, qs)).max(-1)
         kn[:, :, t] = mag / np.where(val > 0, val, 1.0)
+        mabs[:, :, t] = np.abs(mn)
         m = mn
-    return kd, kn
+    return kd, kn, mabs
 
 
 def fp32_row_tolerance(inp, qk_scale=None, heads=None, base=1e-4):
-    """max(base, 32 * 2^-24 * (kappa_den + kappa_num)) per (b, h, t) row."""
-    kd, kn = condition_numbers(inp, qk_scale, heads)
-    return np.maximum(base, 32.0 * 2.0 ** -24 * (kd + kn))
+    """max(base, 32 * 2^-24 * (kappa_den + kappa_num + |m_t|)) per (b, h, t) row.
+
+    The |m_t| term covers the log-space gate arithmetic: exponents such as
+    f~ + m_{t-1} - m_t are formed from numbers of size |m|, so in fp32 they carry
+    an absolute error of about |m| 2^-24, a relative error of the gates."""
+    kd, kn, mabs = condition_numbers(inp, qk_scale, heads)
+    return np.maximum(base, 32.0 * 2.0 ** -24 * (kd + kn + mabs))
 
 
 def compare(got, ref, dtype: str, what: str = "", check_state=True, row_tol=None):

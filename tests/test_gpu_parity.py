@@ -31,7 +31,15 @@ SMALL = [  # B, H, T, dqk, dv
     (2, 1, 130, 128, 32),
     (1, 1, 64, 16, 128),
     (1, 2, 200, 256, 64),
+    # shapes the tensor-core kernel takes for bf16 (d_qk in {64,128,256}, d_v % 128 == 0)
+    (1, 2, 200, 64, 128),
+    (2, 1, 130, 128, 256),
+    (1, 1, 333, 256, 128),
+    (1, 2, 64, 256, 512),
+    (2, 2, 1, 128, 128),
+    (1, 1, 65, 64, 384),
 ]
+TC_SHAPES = [sh for sh in SMALL if sh[3] in (64, 128, 256) and sh[4] % 128 == 0]
 
 
 def small_inputs(B, H, T, dqk, dv, dtype, state, seed=7, gate="std", mean_i=0.0, std_i=1.5):
@@ -53,9 +61,21 @@ def test_small_shapes(kind, dtype, shape, state):
         compare(got, ref, dtype, f"{kind} {dtype} {shape} state={state} scale={scale:.3f}")
 
 
+def test_tensor_core_path_selected():
+    """bf16 inputs of the supported head sizes run on the tcgen05 kernel."""
+    for B, H, T, dqk, dv in TC_SHAPES:
+        d = capi.make_desc(B, H, T, dqk, dv, capi.XLSTM_BF16, 1.0, 64)
+        assert capi.xlstm_mlstm_chunkwise_kernel(d) == "tcgen05", (B, H, T, dqk, dv)
+        d.qkv_dtype = capi.XLSTM_F32
+        assert capi.xlstm_mlstm_chunkwise_kernel(d) == "simt"
+    d = capi.make_desc(8, 8, 4096, 256, 512, capi.XLSTM_BF16, 1 / 16, 64)
+    assert capi.xlstm_mlstm_chunkwise_kernel(d) == "tcgen05"
+
+
+@pytest.mark.parametrize("dv", [64, 128])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_chunk_size_invariance(dtype):
-    inp = small_inputs(2, 2, 203, 64, 64, dtype, True, seed=3)
+def test_chunk_size_invariance(dtype, dv):
+    inp = small_inputs(2, 2, 203, 64, dv, dtype, True, seed=3)
     ref = oracle_sequence(inp)
     outs = {}
     for L in (16, 32, 64):
@@ -67,11 +87,13 @@ def test_chunk_size_invariance(dtype):
         assert mx <= tol, f"chunk {L} vs 64: {mx:.2e}"
 
 
-@pytest.mark.parametrize("gate,mean_i,std_i", [("mixed", 0.0, 1.0), ("std", 4.0, 6.0)])
+@pytest.mark.parametrize("gate,mean_i,std_i", [("mixed", 0.0, 1.0), ("std", 4.0, 6.0), ("std", 30.0, 40.0)])
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_stabilizer_stress(gate, mean_i, std_i, dtype):
-    """Positive log-forget gates (exp(f~) > 1) and large input-gate jumps."""
-    inp = small_inputs(2, 2, 300, 64, 64, dtype, True, seed=11, gate=gate, mean_i=mean_i, std_i=std_i)
+@pytest.mark.parametrize("dv", [64, 128])
+def test_stabilizer_stress(gate, mean_i, std_i, dtype, dv):
+    """Positive log-forget gates (exp(f~) > 1), large input-gate jumps, and
+    jumps far beyond the tensor-core kernel's lazy-rescale threshold."""
+    inp = small_inputs(2, 2, 300, 64, dv, dtype, True, seed=11, gate=gate, mean_i=mean_i, std_i=std_i)
     ref = oracle_sequence(inp)
     tol = fp32_row_tolerance(inp)
     for kind in ("chunkwise", "recurrent"):
@@ -79,9 +101,10 @@ def test_stabilizer_stress(gate, mean_i, std_i, dtype):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_reset_gates(dtype):
+@pytest.mark.parametrize("dv", [64, 128])
+def test_reset_gates(dtype, dv):
     """f~ = -1e4 at every token: each token forgets everything before it."""
-    inp = small_inputs(1, 2, 150, 64, 64, dtype, True, seed=5)
+    inp = small_inputs(1, 2, 150, 64, dv, dtype, True, seed=5)
     inp["f_pre"] = np.full_like(inp["f_pre"], -1.0e4)
     ref = oracle_sequence(inp)
     for kind in ("chunkwise", "recurrent"):
@@ -99,9 +122,10 @@ def test_empty_sequence_passes_state_through():
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_composition_across_calls(dtype):
+@pytest.mark.parametrize("dv", [32, 256])
+def test_composition_across_calls(dtype, dv):
     """run(T1+T2) == run(T2, state=run(T1).state), mixing call types."""
-    inp = small_inputs(2, 2, 150, 64, 32, dtype, True, seed=9)
+    inp = small_inputs(2, 2, 150, 64, dv, dtype, True, seed=9)
     ref = oracle_sequence(inp)
     s = 70
     first = {k: (v[:, :, :s] if k in ("q", "k", "v", "i_pre", "f_pre") else v) for k, v in inp.items()}
@@ -150,6 +174,26 @@ def test_invalid_arguments_rejected():
     assert f(d, q, q, q, g, g, None, None, None, h, None, None, None, ws, 256) == capi.XLSTM_ERR_UNSUPPORTED
     torch.cuda.synchronize()
     assert capi.xlstm_mlstm_workspace_status(ws)[0] == capi.XLSTM_OK
+
+
+def test_device_wait_timeout_reports_status():
+    """A bounded device-side wait that runs out (a hand-off withheld through
+    the test hook) ends the kernel cleanly with XLSTM_ERR_TIMEOUT in the
+    workspace status block; the context stays usable and the next call is
+    correct."""
+    inp = small_inputs(1, 2, 300, 64, 128, "bf16", True, seed=13)
+    q, k, v = (to_dev(inp[n], "bf16") for n in ("q", "k", "v"))
+    ig, fg = to_dev(inp["i_pre"], "f32"), to_dev(inp["f_pre"], "f32")
+    st = tuple(to_dev(inp[n], "f32") for n in ("C0", "n0", "m0"))
+    ws = torch.zeros(256, device="cuda", dtype=torch.uint8)
+    capi.xlstm_mlstm_test_timeout_next(1)
+    capi.fwd(q, k, v, ig, fg, state=st, qk_scale=inp["qk_scale"], workspace=ws)
+    status, where = capi.xlstm_mlstm_workspace_status(ws)
+    assert status == capi.XLSTM_ERR_TIMEOUT and where > 0, (status, where)
+    h, (C, n, m) = capi.fwd(q, k, v, ig, fg, state=st, qk_scale=inp["qk_scale"], workspace=ws)
+    assert capi.xlstm_mlstm_workspace_status(ws)[0] == capi.XLSTM_OK
+    compare((h.cpu().numpy(), C.cpu().numpy(), n.cpu().numpy(), m.cpu().numpy()),
+            oracle_sequence(inp), "bf16", "after timeout")
 
 
 # ---- full-size workloads, sampled heads ------------------------------------------

@@ -20,7 +20,7 @@ XLSTM_F32, XLSTM_BF16 = 0, 1
 
 EXPORTED = ("xlstm_mlstm_fwd_chunkwise", "xlstm_mlstm_fwd_recurrent", "xlstm_mlstm_step",
             "xlstm_mlstm_workspace_size", "xlstm_mlstm_workspace_status", "xlstm_status_string",
-            "xlstm_mlstm_version")
+            "xlstm_mlstm_version", "xlstm_mlstm_chunkwise_kernel", "xlstm_mlstm_test_timeout_next")
 
 
 class xlstm_mlstm_desc_t(ctypes.Structure):
@@ -62,6 +62,10 @@ def load(path: str = LIB_PATH):
     lib.xlstm_status_string.restype = ctypes.c_char_p
     lib.xlstm_mlstm_version.argtypes = []
     lib.xlstm_mlstm_version.restype = ctypes.c_char_p
+    lib.xlstm_mlstm_chunkwise_kernel.argtypes = [dp]
+    lib.xlstm_mlstm_chunkwise_kernel.restype = ctypes.c_char_p
+    lib.xlstm_mlstm_test_timeout_next.argtypes = [ctypes.c_int32]
+    lib.xlstm_mlstm_test_timeout_next.restype = None
     if path == LIB_PATH:
         _lib = lib
     return lib
@@ -129,6 +133,14 @@ def xlstm_status_string(status: int) -> str:
 
 def xlstm_mlstm_version() -> str:
     return load().xlstm_mlstm_version().decode()
+
+
+def xlstm_mlstm_chunkwise_kernel(desc) -> str:
+    return load().xlstm_mlstm_chunkwise_kernel(ctypes.byref(desc)).decode()
+
+
+def xlstm_mlstm_test_timeout_next(enable: int = 1) -> None:
+    load().xlstm_mlstm_test_timeout_next(int(enable))
 
 
 def status_string(status: int) -> str:

@@ -190,4 +190,16 @@ const char *xlstm_status_string(xlstm_status_t s) {
 
 const char *xlstm_mlstm_version(void) { return "xlstm_mlstm_b200 0.1 (sm_100a)"; }
 
+const char *xlstm_mlstm_chunkwise_kernel(const xlstm_mlstm_desc_t *desc) {
+    if (!desc || !dims_ok(desc)) return "none";
+    const int L = desc->chunk ? desc->chunk : 64;
+    if (L != 16 && L != 32 && L != 64) return "none";
+    FwdArgs a = pack(desc, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                     nullptr, nullptr, nullptr, nullptr);
+    if (a.T == 0) return "copy";
+    return xlstm::chunkwise_tc_supported(a) ? "tcgen05" : "simt";
+}
+
+void xlstm_mlstm_test_timeout_next(int32_t enable) { xlstm::set_chunkwise_tc_fault(enable ? 1 : 0); }
+
 }  // extern "C"

@@ -10,6 +10,9 @@
 //          / max(|e^{m0-mu_t} n~0.q_t + sum_{s<=t} e^{u_s-mu_t} q_t.k_s|, e^{-m_t}),
 //   C~_L = e^{m0-mu_L} C~0 + sum_s e^{u_s-mu_L} v_s k_s^T  (likewise n~), m <- m_L.
 // Every exponent above is <= 0, so nothing overflows however large the gates.
+// The gate scan runs in float64 and hands the pairwise exponents u_s - mu_t on
+// as float hi/lo pairs: with strong forgetting F_t reaches 1e5 and more inside
+// one chunk, where the fp32 difference would cancel catastrophically.
 //
 // A block owns kDvs rows of C~ for one (batch, head) and keeps them in shared
 // memory for the whole sequence; q and k are streamed through in kKt-wide
@@ -33,7 +36,9 @@ struct ChunkP {
 
 template <typename Tin, int L>
 __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkP p) {
-    extern __shared__ float sm[];
+    extern __shared__ double smd[];
+    double *mst = smd;                       // carried stabilizer m (float64)
+    float *sm = reinterpret_cast<float *>(smd + 2);
     const int dqk = p.dqk, dv = p.dv;
     const int cst = dqk + 1;                 // padded row stride of C~
     float *Cs = sm;                          // [kDvs][dqk+1]
@@ -43,9 +48,9 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkP p) {
     float *Vs = Kt + L * (kKt + 1);          // [L][kDvs]
     float *Ps = Vs + L * kDvs;               // [L][L+1]
     float *sc = Ps + L * (L + 1);            // per-token scalars
-    float *u_s = sc, *mu_s = sc + L, *al_s = sc + 2 * L, *lo_s = sc + 3 * L;
-    float *g_s = sc + 4 * L, *nq_s = sc + 5 * L, *r_s = sc + 6 * L, *ig_s = sc + 7 * L,
-          *fg_s = sc + 8 * L, *misc = sc + 9 * L;   // misc[0] = beta, misc[1] = m
+    float *uh_s = sc, *ul_s = sc + L, *mh_s = sc + 2 * L, *ml_s = sc + 3 * L, *al_s = sc + 4 * L;
+    float *lo_s = sc + 5 * L, *g_s = sc + 6 * L, *nq_s = sc + 7 * L, *r_s = sc + 8 * L;
+    float *ig_s = sc + 9 * L, *fg_s = sc + 10 * L, *misc = sc + 11 * L;   // misc[0] = beta, misc[1] = m
 
     const int bh = blockIdx.x / p.slices;
     const int row0 = (blockIdx.x % p.slices) * kDvs;
@@ -59,7 +64,10 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkP p) {
         Cs[r * cst + j] = (p.C0 && row0 + r < dv) ? p.C0[((size_t)bh * dv + row0 + r) * dqk + j] : 0.f;
     }
     for (int j = tid; j < dqk; j += kThreads) ns[j] = p.n0 ? p.n0[(size_t)bh * dqk + j] : 0.f;
-    if (tid == 0) misc[1] = p.m0 ? p.m0[bh] : 0.f;
+    if (tid == 0) {
+        mst[0] = p.m0 ? (double)p.m0[bh] : 0.0;
+        misc[1] = (float)mst[0];
+    }
 
     constexpr int kS = (L * L + kThreads - 1) / kThreads;     // S entries per thread
     constexpr int kH = (L * kDvs + kThreads - 1) / kThreads;  // h entries per thread
@@ -72,22 +80,29 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkP p) {
             fg_s[tid] = tid < len ? p.fg[(size_t)bh * p.T + t0 + tid] : 0.f;
         }
         __syncthreads();
-        if (tid == 0) {   // gate scan: cumulative log forget and running max
-            const float m0 = misc[1];
-            float F = 0.f, mu = m0;
+        if (tid == 0) {   // gate scan (float64): cumulative log forget and running max
+            const double m0 = mst[0];
+            double F = 0.0, mu = m0;
             for (int t = 0; t < len; ++t) {
-                F += fg_s[t];
-                const float u = ig_s[t] - F;
-                mu = fmaxf(mu, u);
-                u_s[t] = u;
-                mu_s[t] = mu;
-                al_s[t] = expf(m0 - mu);
-                lo_s[t] = expf(-(F + mu));
+                F += (double)fg_s[t];
+                const double u = (double)ig_s[t] - F;
+                mu = fmax(mu, u);
+                uh_s[t] = (float)u;
+                ul_s[t] = isfinite(uh_s[t]) ? (float)(u - (double)uh_s[t]) : 0.f;
+                mh_s[t] = (float)mu;
+                ml_s[t] = (float)(mu - (double)mh_s[t]);
+                al_s[t] = expf((float)(m0 - mu));
+                lo_s[t] = expf((float)(-(F + mu)));
             }
-            for (int t = 0; t < len; ++t) g_s[t] = expf(u_s[t] - mu);
-            for (int t = len; t < L; ++t) { u_s[t] = 0.f; mu_s[t] = mu; al_s[t] = 0.f; lo_s[t] = 1.f; g_s[t] = 0.f; }
-            misc[0] = expf(m0 - mu);
-            misc[1] = F + mu;
+            for (int t = 0; t < len; ++t)
+                g_s[t] = expf((float)(((double)uh_s[t] + (double)ul_s[t]) - mu));
+            for (int t = len; t < L; ++t) {
+                uh_s[t] = 0.f; ul_s[t] = 0.f; mh_s[t] = 0.f; ml_s[t] = 0.f;
+                al_s[t] = 0.f; lo_s[t] = 1.f; g_s[t] = 0.f;
+            }
+            misc[0] = expf((float)(m0 - mu));
+            mst[0] = F + mu;
+            misc[1] = (float)mst[0];
         }
 
         // S = Q K^T, H_inter = Q C~0^T, nq = Q n~0, over d_qk tiles.
@@ -138,7 +153,8 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkP p) {
             const int e = tid + x * kThreads;
             if (e < L * L) {
                 const int t = e / L, s = e % L;
-                Ps[t * (L + 1) + s] = (s <= t && t < len) ? S[x] * expf(u_s[s] - mu_s[t]) : 0.f;
+                const float e = (uh_s[s] - mh_s[t]) + (ul_s[s] - ml_s[t]);
+                Ps[t * (L + 1) + s] = (s <= t && t < len) ? S[x] * expf(e) : 0.f;
             }
         }
         if (tid < L) nq_s[tid] = nq;
@@ -205,8 +221,8 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkP p) {
 
 template <typename Tin, int L>
 cudaError_t launch_L(const ChunkP &p, cudaStream_t s) {
-    const size_t smem = (size_t)(kDvs * (p.dqk + 1) + p.dqk + 2 * L * (kKt + 1) + L * kDvs +
-                                 L * (L + 1) + 9 * L + 2) * sizeof(float);
+    const size_t smem = 2 * sizeof(double) + (size_t)(kDvs * (p.dqk + 1) + p.dqk + 2 * L * (kKt + 1) +
+                                                      L * kDvs + L * (L + 1) + 11 * L + 2) * sizeof(float);
     auto kern = chunk_simt_kernel<Tin, L>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;

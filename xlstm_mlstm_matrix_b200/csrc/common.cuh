@@ -29,6 +29,7 @@ cudaError_t launch_recurrent(const FwdArgs &a, cudaStream_t s);
 cudaError_t launch_chunkwise_simt(const FwdArgs &a, cudaStream_t s);
 bool chunkwise_tc_supported(const FwdArgs &a);
 cudaError_t launch_chunkwise_tc(const FwdArgs &a, cudaStream_t s);
+void set_chunkwise_tc_fault(int mode);   // test hook: applies to the next launch only
 
 // ---- small device helpers ------------------------------------------------
 __device__ __forceinline__ float to_f32(float x) { return x; }
