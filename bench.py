@@ -198,6 +198,8 @@ def run_ours(args, rank, world, local_rank):
     torch.cuda.set_device(dev)
     capi.load()
     w = inputs.WORKLOADS[WORKLOAD].replace(seed=inputs.WORKLOADS[WORKLOAD].seed + 1000 * rank)
+    if args.B or args.H:   # smaller batch/head count of the same layer (profiling captures)
+        w = w.replace(B=args.B or w.B, H=args.H or w.H)
     inp = inputs.make_sequence(w)
     scale = inp["qk_scale"]
     desc = capi.make_desc(w.B, w.H, w.T, w.d_qk, w.d_v, capi.XLSTM_BF16, scale, 64)
@@ -291,18 +293,19 @@ def run_ours(args, rank, world, local_rank):
         for dst, src in ((oh, h), (oC, C1), (on, n1), (om, m1)):
             dst.copy_(src, non_blocking=True)
 
-    e2e_steps = max(1, min(args.steps, 5))
-    with torch.cuda.stream(stream):
-        e2e_step()
-        stream.synchronize()
-        barrier()
-        e0.record(stream)
-        for _ in range(e2e_steps):
+    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 5))
+    if e2e_steps:
+        with torch.cuda.stream(stream):
             e2e_step()
-        e1.record(stream)
-        e1.synchronize()
-    barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps)
+            stream.synchronize()
+            barrier()
+            e0.record(stream)
+            for _ in range(e2e_steps):
+                e2e_step()
+            e1.record(stream)
+            e1.synchronize()
+        barrier()
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps) if e2e_steps else None
 
     if rank == 0:
         line = {
@@ -321,8 +324,9 @@ def run_ours(args, rank, world, local_rank):
                          "algorithmic_bytes_per_launch": bytes_, "flops_per_launch": flops,
                          "tensor_frac": flops / (ms * 1e-3) / 1e12 / bf16_peak},
             "gpu_launches": args.steps,
-            "e2e": {"value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT,
-                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "e2e": None if e2e_ms is None else {
+                "value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "clocks": clk.summary(),
             "kernel_source_sha": src_sha,
         }
@@ -339,6 +343,9 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--ref-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
+    ap.add_argument("--H", type=int, default=0, help="override the head count (profiling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank = int(os.environ.get("RANK", 0))

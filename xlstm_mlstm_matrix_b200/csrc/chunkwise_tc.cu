@@ -4,38 +4,45 @@
 // stabilizer), evaluated per chunk of L = 64 tokens.  With the chunk-local
 // cumulative log forget gate F_t = sum_{r<=t} f~_r, u_s = i~_s - F_s and the
 // running maximum mu_t = max(m, max_{s<=t} u_s), the stabilizer is exactly
-// m_t = F_t + mu_t, and
+// m_t = F_t + mu_t, and (q already multiplied by qk_scale)
 //   h~_t = [e^{b-mu_t} C_acc q_t + sum_{s<=t} e^{u_s-mu_t} (q_t.k_s) v_s]
-//          / max(|e^{b-mu_t} n_acc.q_t + sum_{s<=t} e^{u_s-mu_t} q_t.k_s|, e^{-m_t})
-// (q already multiplied by qk_scale).  (C_acc, n_acc) is the state in a lazily
-// moved gauge, C~ = e^{b-m} C_acc with b <= m.  The update is
-//   C_acc <- e^{b-b'} C_acc + sum_s e^{u_s-b'} v_s k_s^T
-// with b' = b (weights <= e^{kRescale}) unless the stabilizer ran more than
-// kRescale past b; then b' = mu_L and C_acc is rescaled once in tensor memory.
-// Every exponent is <= 0 except those bounded update weights.  The gate scan
-// runs in float64 (one warp, 64 tokens per chunk): with strong forgetting F_t
-// reaches 1e5 and more inside one chunk, where m_t = F_t + mu_t and the
-// pairwise exponents u_s - mu_t would otherwise cancel catastrophically in
-// fp32; the pairwise exponents are handed on as float hi/lo pairs.
+//          / max(|e^{b-mu_t} n_acc.q_t + sum_{s<=t} e^{u_s-mu_t} q_t.k_s|, e^{-m_t}).
+// (C_acc, n_acc) is the state in a lazily moved gauge: C~ = e^{b-m} C_acc, b <= m.
 //
-// Block = one (batch, head) and a 128-row slice of d_v; it walks the chunks in
-// order with C_acc (128 x d_qk fp32) resident in tensor memory.  Per chunk:
-//   S       = Q K^T                           kind::f16 M=64  N=64 K=d_qk
-//   H_inter = (C_hi + C_lo) Q^T               kind::f16 M=128 N=64 K=d_qk, A in TMEM
-//   H_intra = V^T (P_hi + P_lo)^T             kind::f16 M=128 N=64 K=64
-//   C_acc  += (w V)^T K                       kind::f16 M=128 N=d_qk K=64
-// C_hi = bf16(C_acc), C_lo = bf16(C_acc - C_hi) (a 16-bit split, ~2^-17
-// relative) are written each chunk by the CUDA-core warps; the same split is
-// used for P_ts = scale S_ts e^{u_s-mu_t} [s<=t].  A single bf16 or tf32 copy
-// of either loses up to 2^-9 / 2^-11 per element, which rows whose readout
-// cancels amplify past a 2e-2 tolerance.  q itself is bf16 and exact, so the
-// readout multiplies the raw q tile; e^{b-mu_t} scale is applied per token in
-// the epilogue:  h~[t][v] = (a_t H_inter[v][t] + H_intra[v][t]) / den_t.
+// Each chunk picks a reference r (>= b) and weights w_s = e^{u_s-r}:
+//   fast chunk (the stabilizer rises by at most kGrowth inside the chunk):
+//     r = b if mu_L - b <= kRescale, else mu_L - kRescale (the state is then
+//     rescaled by rho = e^{b-r} as it is split).  Because e^{u_s-mu_t} =
+//     w_s e^{r-mu_t}, one accumulator holds the whole numerator,
+//        H = (rho C_acc) Q^T + (w V)^T (mask S)^T,    h~_t = a_t H_t / den_t,
+//     with a_t = scale e^{r-mu_t} <= scale e^{kGrowth-kRescale}, w_s <= e^{kRescale}:
+//     no per-element exponentials and no overflow.
+//   exact chunk (the stabilizer jumps by more, e.g. a forget gate near zero):
+//     r = mu_L, P_ts = scale S_ts e^{u_s-mu_t} element by element (every
+//     exponent <= 0), the intra part kept in its own accumulator.
+// The update is C_acc <- rho C_acc + (w V)^T K, b <- r + F_L.  The gate scan runs
+// in float64 (one warp): inside a chunk F_t can reach 1e5 (strong forgetting),
+// where m_t = F_t + mu_t and u_s - mu_t would cancel in fp32; pairwise
+// exponents are handed on as float hi/lo pairs.
 //
-// Warp roles: 0 TMA producer, 1 MMA issuer (and TMEM owner), 2 gate scan,
-// 3 normaliser n_acc, 4-7 state split, P, epilogue.  Every wait is bounded: a
-// wait that gives up records XLSTM_ERR_TIMEOUT in the status block, each role
-// drains what it has in flight, tensor memory is freed and the kernel returns.
+// Block = one (batch, head) and 128 value rows; C_acc (128 x d_qk fp32) lives in
+// tensor memory for the whole sequence.  Per chunk, on the tensor cores:
+//   S   = Q K^T                          kind::f16 M=64  N=64 K=d_qk
+//   H   = (C_hi + C_lo) Q^T              kind::f16 M=128 N=64 K=d_qk (C_hi from TMEM)
+//   H  += (w V)^T (P_hi + P_lo)^T        kind::f16 M=128 N=64 K=64
+//   C_acc += (w V)^T K                   kind::f16 M=128 N=d_qk K=64
+// C_hi = bf16(C), C_lo = bf16(C - C_hi) and the same split of P give ~2^-17
+// relative operands: a single bf16 or tf32 copy loses 2^-9 / 2^-11 per element,
+// which rows whose readout or normaliser cancels amplify past 2e-2.  q is bf16
+// and exact, so the raw q tile is the readout operand.  For d_qk = 256 tensor
+// memory is full (C_acc 256 + C_hi 128 + H 64 + S 64 columns) and C_lo goes
+// through a 32 KB shared half-buffer, refilled while the first half is read.
+//
+// Warps: 0 TMA producer, 1 MMA issuer (owns TMEM), 2 gate scan, 3 normaliser,
+// 4-7 state group (lower half of the state split, epilogue), 8-11 token group
+// (w V, upper half of the state split, n.q, P).
+// Every wait is bounded: one that gives up records XLSTM_ERR_TIMEOUT in the
+// status block; each role drains what it has in flight, TMEM is freed, return.
 #include <math.h>
 
 #include "common.cuh"
@@ -48,19 +55,20 @@ namespace {
 using namespace sm100;
 
 constexpr int kL = 64;              // chunk length
-constexpr int kDvs = 128;           // rows of C per block
-constexpr int kThreads = 256;
+constexpr int kDvs = 128;           // value rows per block
+constexpr int kThreads = 384;
 constexpr int kNG = 4;              // gate-ring slots
-constexpr double kRescale = 20.0;   // gauge drift allowed before C_acc is rescaled
+constexpr double kRescale = 20.0;   // gauge drift allowed before the state is rescaled
+constexpr double kGrowth = 90.0;    // stabilizer rise inside a chunk handled by the fast path
 constexpr double kLog2e = 1.4426950408889634;
 constexpr uint64_t kTimeoutNs = 1000000000ull;   // 1 s per wait
 
 // Where a wait gave up (reported in the status block).
 enum : int32_t {
-    kWhereTmaKvEmpty = 1, kWhereTmaQEmpty, kWhereMmaKvFull, kWhereMmaQFull, kWhereMmaSEmpty,
-    kWhereMmaOps, kWhereMmaHEmpty, kWhereMmaUpd, kWhereGateEmpty, kWhereNormGate, kWhereNormKv,
-    kWhereNormFree, kWhereCwGate, kWhereCwQ, kWhereCwN, kWhereCwS, kWhereCwH, kWhereCwFinal,
-    kWhereCwUpd, kWhereMmaConv
+    kWhereTmaKvEmpty = 1, kWhereTmaQEmpty, kWhereMmaKvFull, kWhereMmaQFull, kWhereMmaSEmpty, kWhereMmaGate,
+    kWhereMmaConv, kWhereMmaOps, kWhereMmaVt, kWhereMmaHEmpty, kWhereMmaClo, kWhereGateEmpty, kWhereNormGate,
+    kWhereNormKv, kWhereNormFree, kWhereStUpd, kWhereStGate, kWhereStClo, kWhereStOps, kWhereStH, kWhereStFinal,
+    kWhereTkH, kWhereTkGate, kWhereTkKv, kWhereTkQ, kWhereTkN, kWhereTkS, kWhereTkUpd, kWhereTkClo
 };
 
 // Test hook: make the gate warp withhold one hand-off so that its consumers time out.
@@ -72,25 +80,24 @@ namespace {
 
 template <int DQK>
 struct Cfg {
-    static constexpr bool BIG = DQK == 256;            // TMEM is full: C_lo in smem, S shares H_intra
+    static constexpr bool BIG = DQK == 256;
     static constexpr int NKB = DQK / 64;               // 64-column boxes of q and k
-    static constexpr int QST = BIG ? 1 : 2;            // q stages
     static constexpr int Q_BYTES = NKB * 8192;
     static constexpr int K_BYTES = NKB * 8192;
     static constexpr int V_BYTES = 2 * 8192;           // 128 value columns
     static constexpr int P_BYTES = 2 * 8192;           // P_hi, P_lo
-    static constexpr int CLO_BYTES = BIG ? NKB * 16384 : 0;   // 128 rows x d_qk bf16
-    static constexpr int OFF_Q = 0;
-    static constexpr int OFF_K = OFF_Q + QST * Q_BYTES;
+    static constexpr int CLO_BYTES = BIG ? 2 * 16384 : 0;     // half of C_lo: 128 rows x 128 cols bf16
+    static constexpr int OFF_Q = 0;                    // two stages each
+    static constexpr int OFF_K = OFF_Q + 2 * Q_BYTES;
     static constexpr int OFF_V = OFF_K + 2 * K_BYTES;
     static constexpr int OFF_P = OFF_V + 2 * V_BYTES;
     static constexpr int OFF_CLO = OFF_P + P_BYTES;
-    // gate ring: per slot UH, UL, MH, ML, A, W, LOWER [64] + 8 chunk scalars
-    static constexpr int G_FLOATS = 7 * kL + 8;
+    // gate ring: per slot UH, UL, MH, ML, AH, AN, W, LOWER [64] + 8 chunk scalars
+    static constexpr int G_FLOATS = 8 * kL + 8;
     static constexpr int OFF_G = OFF_CLO + CLO_BYTES;
     static constexpr int OFF_N = OFF_G + kNG * G_FLOATS * 4;   // n_acc double buffer
-    static constexpr int OFF_SC = OFF_N + 2 * DQK * 4;          // nq, rsum, inv_den [64]
-    static constexpr int OFF_BAR = OFF_SC + 3 * kL * 4;
+    static constexpr int OFF_SC = OFF_N + 2 * DQK * 4;          // nq, rsum, inv, coef [2][64] each
+    static constexpr int OFF_BAR = OFF_SC + 8 * kL * 4;
     static constexpr int NBARS = 32;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM = OFF_MISC + 64 + 1024;          // + alignment slack
@@ -98,26 +105,24 @@ struct Cfg {
     static constexpr uint32_t TM_C = 0;
     static constexpr uint32_t TM_CHI = DQK;
     static constexpr uint32_t TM_CLO = DQK + DQK / 2;          // unused when BIG
-    static constexpr uint32_t TM_HI = BIG ? DQK + DQK / 2 : 2 * DQK;
-    static constexpr uint32_t TM_HA = TM_HI + 64;
-    static constexpr uint32_t TM_S = BIG ? TM_HA : TM_HA + 64;
+    static constexpr uint32_t TM_H = BIG ? DQK + DQK / 2 : 2 * DQK;
+    static constexpr uint32_t TM_S = TM_H + 64;                // S, or the intra part of an exact chunk
     static_assert(TM_S + 64 <= TMEM_COLS, "tensor memory budget");
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
-// Gate-ring slot field offsets (floats).
+// Gate-ring slot fields (floats).
 enum : int {
-    kGUh = 0, kGUl = kL, kGMh = 2 * kL, kGMl = 3 * kL, kGA = 4 * kL, kGW = 5 * kL, kGLower = 6 * kL,
-    kGScal = 7 * kL
+    kGUh = 0, kGUl = kL, kGMh = 2 * kL, kGMl = 3 * kL, kGAH = 4 * kL, kGAN = 5 * kL, kGW = 6 * kL,
+    kGLower = 7 * kL, kGScal = 8 * kL
 };
-// Chunk scalars inside a slot.
-enum : int { kSRho = 0, kSRescale = 1, kSMEnd = 2, kSGsc = 3 };
+enum : int { kSRho = 0, kSRescale = 1, kSExact = 2, kSMEnd = 3, kSGsc = 4 };
 
-// Barrier indices.
+// Barriers.
 enum : int {
     B_KV_FULL = 0, B_KV_EMPTY = 2, B_Q_FULL = 4, B_Q_EMPTY = 6, B_G_FULL = 8, B_G_EMPTY = B_G_FULL + kNG,
-    B_S_FULL = B_G_EMPTY + kNG, B_S_EMPTY, B_OPS, B_CONV, B_H_FULL, B_H_EMPTY, B_UPD_READY, B_UPD_DONE,
-    B_N_READY, B_N_FREE = B_N_READY + 2, B_DRAIN = B_N_FREE + 2, B_COUNT
+    B_S_FULL = B_G_EMPTY + kNG, B_S_EMPTY, B_OPS, B_VT, B_CONV0, B_CONV1, B_CLO_FREE, B_H_FULL, B_H_EMPTY,
+    B_UPD_DONE, B_N_READY, B_N_FREE = B_N_READY + 2, B_DRAIN = B_N_FREE + 2, B_COUNT
 };
 static_assert(B_COUNT <= 32, "barrier space");
 
@@ -146,7 +151,8 @@ __device__ __forceinline__ bool wait1(const Shared &sh, uint64_t *bar, uint32_t 
     if (mbar_try_wait(bar, parity)) return true;
     const uint64_t t0 = global_timer_ns();
     for (;;) {
-        if (mbar_try_wait(bar, parity)) return true;
+        // suspended in hardware (no issue slots) until the phase completes or 20 us pass
+        if (mbar_try_wait_suspend(bar, parity, 20000)) return true;
         if (*sh.abort_flag) return false;
         if (global_timer_ns() - t0 > kTimeoutNs) {
             record_timeout(sh, where);
@@ -180,10 +186,91 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
 __device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
+// (x0, x1) -> bf16 pairs hi = trunc(x), lo = round(x - hi): |x - hi - lo| <= 2^-16 |x|.
+// The high half is a plain truncation (two masks and a byte permute) so that
+// only the residual needs a rounding conversion.
+__device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, uint32_t &lo) {
+    const uint32_t a = __float_as_uint(x0), b = __float_as_uint(x1);
+    hi = __byte_perm(a, b, 0x7632);
+    const float2 r = __fadd2_rn(make_float2(x0, x1), make_float2(__uint_as_float((a & 0xFFFF0000u) ^ 0x80000000u),
+                                                                __uint_as_float((b & 0xFFFF0000u) ^ 0x80000000u)));
+    lo = pack_bf16x2(r.x, r.y);
+}
+__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u) {
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
+}
+
 // x -> (hi, lo) float pair with hi + lo = x to ~2^-48; -inf -> (-inf, 0).
 __device__ __forceinline__ void split_double(double x, float &hi, float &lo) {
     hi = (float)x;
     lo = isfinite(hi) ? (float)(x - (double)hi) : 0.f;
+}
+
+// V <- w V in place: 1024 16-byte chunks of a 64-token x 128-value stage, chunk
+// e in row (token) (e mod 512) / 8; 128 threads, 8 chunks each.
+// All loads are issued before any store: the stores go to the same buffer, so
+// interleaving them would serialise every load behind the previous store.
+__device__ __forceinline__ void scale_v_rows(uint8_t *Vs, const float *w, int t128) {
+    uint4 u[8];
+    float ws[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = t128 + 128 * i;
+        u[i] = *reinterpret_cast<const uint4 *>(Vs + 16 * e);
+        ws[i] = w[(e & 511) >> 3];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float2 w2 = make_float2(ws[i], ws[i]);
+        const float2 a = __fmul2_rn(bf16x2_to_float2(u[i].x), w2), b = __fmul2_rn(bf16x2_to_float2(u[i].y), w2);
+        const float2 c = __fmul2_rn(bf16x2_to_float2(u[i].z), w2), d = __fmul2_rn(bf16x2_to_float2(u[i].w), w2);
+        u[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(b.x, b.y), pack_bf16x2(c.x, c.y), pack_bf16x2(d.x, d.y));
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4 *>(Vs + 16 * (t128 + 128 * i)) = u[i];
+}
+
+// 32 consecutive floats of a shared array into registers (broadcast loads).
+__device__ __forceinline__ void load32(const float *src, float (&d)[32]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float4 x = reinterpret_cast<const float4 *>(src)[i];
+        d[4 * i] = x.x; d[4 * i + 1] = x.y; d[4 * i + 2] = x.z; d[4 * i + 3] = x.w;
+    }
+}
+
+// One 32-column block [32 i, 32 i + 32) of this thread's C_acc row: optional
+// gauge move (C_acc *= rho, written back), then the split C = C_hi + C_lo.
+// lo_mode: 0 C_hi and C_lo to TMEM; 1 C_hi to TMEM, C_lo to the shared tile at
+// local column jlo; 2 C_hi only; 3 C_lo only (shared tile, no gauge move).
+template <class C>
+__device__ __forceinline__ void split_state_block(uint32_t tm, uint32_t lane_base, int i, bool mv, float rho,
+                                                  int lo_mode, uint8_t *clo_s, int row, int jlo) {
+    float r[32];
+    tmem_ld32(tm + lane_base + C::TM_C + 32 * i, r);
+    tmem_wait_ld();
+    if (mv) {
+#pragma unroll
+        for (int x = 0; x < 32; x += 2) {
+            const float2 y = __fmul2_rn(make_float2(r[x], r[x + 1]), make_float2(rho, rho));
+            r[x] = y.x; r[x + 1] = y.y;
+        }
+        tmem_st32(tm + lane_base + C::TM_C + 32 * i, r);
+    }
+    uint32_t hi[16], lo[16];
+#pragma unroll
+    for (int x = 0; x < 16; ++x) split_bf16x2(r[2 * x], r[2 * x + 1], hi[x], lo[x]);
+    if (lo_mode != 3) tmem_st16(tm + lane_base + C::TM_CHI + 16 * i, hi);
+    if (lo_mode == 0) {
+        tmem_st16(tm + lane_base + C::TM_CLO + 16 * i, lo);
+    } else if (lo_mode == 1 || lo_mode == 3) {   // K-major 128B-swizzled [128 rows][128 cols] bf16 half tile
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+            const int j = jlo + 8 * q4;
+            *reinterpret_cast<uint4 *>(clo_s + (j >> 6) * 16384 + sw128_offset(row, (j & 63) >> 3)) =
+                make_uint4(lo[4 * q4], lo[4 * q4 + 1], lo[4 * q4 + 2], lo[4 * q4 + 3]);
+        }
+    }
 }
 
 template <int DQK>
@@ -198,9 +285,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     Shared sh{reinterpret_cast<volatile int *>(sm + C::OFF_MISC + 4), p.status};
     float *gring = reinterpret_cast<float *>(sm + C::OFF_G);
     float *nbuf = reinterpret_cast<float *>(sm + C::OFF_N);
-    float *nq_s = reinterpret_cast<float *>(sm + C::OFF_SC);
-    float *rs_s = nq_s + kL;
-    float *inv_s = rs_s + kL;
+    float *nq_s = reinterpret_cast<float *>(sm + C::OFF_SC);   // [2][64]
+    float *rs_s = nq_s + 2 * kL;                               // [2][64]
+    float *inv_s = rs_s + 2 * kL;                              // [2][64] 1/den_t
+    float *coef_s = inv_s + 2 * kL;                            // [2][64] AH_t/den_t
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int bh = blockIdx.x / p.nslices;
@@ -215,10 +303,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar[B_Q_FULL + i], 1); mbar_init(&bar[B_Q_EMPTY + i], 2);
             mbar_init(&bar[B_N_READY + i], 1); mbar_init(&bar[B_N_FREE + i], 1);
         }
-        for (int i = 0; i < kNG; ++i) { mbar_init(&bar[B_G_FULL + i], 1); mbar_init(&bar[B_G_EMPTY + i], 2); }
-        mbar_init(&bar[B_S_FULL], 1); mbar_init(&bar[B_S_EMPTY], 1); mbar_init(&bar[B_OPS], 1);
-        mbar_init(&bar[B_CONV], 1); mbar_init(&bar[B_H_FULL], 1); mbar_init(&bar[B_H_EMPTY], 1);
-        mbar_init(&bar[B_UPD_READY], 1); mbar_init(&bar[B_UPD_DONE], 1); mbar_init(&bar[B_DRAIN], 1);
+        for (int i = 0; i < kNG; ++i) { mbar_init(&bar[B_G_FULL + i], 1); mbar_init(&bar[B_G_EMPTY + i], 3); }
+        const int ones[] = {B_S_FULL, B_S_EMPTY, B_OPS, B_VT, B_CONV1, B_CLO_FREE, B_H_FULL, B_H_EMPTY,
+                            B_UPD_DONE, B_DRAIN};
+        mbar_init(&bar[B_CONV0], 2);   // both compute groups split half of the state
+        for (int b : ones) mbar_init(&bar[b], 1);
         *sh.abort_flag = 0;
         fence_mbar_init();
         tma_prefetch_desc(&tmq); tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmv);
@@ -238,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) {
             int kv_issued[2] = {0, 0}, q_issued[2] = {0, 0};
             for (int c = 0; c < NC; ++c) {
-                const int s = c & 1, qs = c % C::QST;
+                const int s = c & 1;
                 if (c >= 2 && !wait1(sh, &bar[B_KV_EMPTY + s], ((c >> 1) - 1) & 1, kWhereTmaKvEmpty)) break;
                 mbar_arrive_expect_tx(&bar[B_KV_FULL + s], C::K_BYTES + C::V_BYTES);
                 uint8_t *Ks = sm + C::OFF_K + s * C::K_BYTES;
@@ -246,11 +335,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int b = 0; b < C::NKB; ++b) tma_load_3d(Ks + b * 8192, &tmk, &bar[B_KV_FULL + s], 64 * b, kL * c, bh);
                 for (int b = 0; b < 2; ++b) tma_load_3d(Vs + b * 8192, &tmv, &bar[B_KV_FULL + s], v0 + 64 * b, kL * c, bh);
                 ++kv_issued[s];
-                if (c >= C::QST && !wait1(sh, &bar[B_Q_EMPTY + qs], ((c / C::QST) - 1) & 1, kWhereTmaQEmpty)) break;
-                mbar_arrive_expect_tx(&bar[B_Q_FULL + qs], C::Q_BYTES);
-                uint8_t *Qs = sm + C::OFF_Q + qs * C::Q_BYTES;
-                for (int b = 0; b < C::NKB; ++b) tma_load_3d(Qs + b * 8192, &tmq, &bar[B_Q_FULL + qs], 64 * b, kL * c, bh);
-                ++q_issued[qs];
+                if (c >= 2 && !wait1(sh, &bar[B_Q_EMPTY + s], ((c >> 1) - 1) & 1, kWhereTmaQEmpty)) break;
+                mbar_arrive_expect_tx(&bar[B_Q_FULL + s], C::Q_BYTES);
+                uint8_t *Qs = sm + C::OFF_Q + s * C::Q_BYTES;
+                for (int b = 0; b < C::NKB; ++b) tma_load_3d(Qs + b * 8192, &tmq, &bar[B_Q_FULL + s], 64 * b, kL * c, bh);
+                ++q_issued[s];
             }
             // drain: every issued copy must land before shared memory is released
             for (int s = 0; s < 2; ++s) {
@@ -266,16 +355,16 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t idPV = make_idesc(128, 64, kFmtBF16, kFmtBF16, 1, 0);
             const uint32_t idU = make_idesc(128, DQK, kFmtBF16, kFmtBF16, 1, 1);
             const uint32_t p_addr = smem_u32(Ps), clo_addr = smem_u32(sm + C::OFF_CLO);
-            bool issued = false;
+            bool issued = false, prev_exact = false;
             for (int c = 0; c < NC; ++c) {
-                const int s = c & 1, qs = c % C::QST;
-                const uint32_t q_addr = smem_u32(sm + C::OFF_Q + qs * C::Q_BYTES);
+                const int s = c & 1, slot = c % kNG;
+                const uint32_t q_addr = smem_u32(sm + C::OFF_Q + s * C::Q_BYTES);
                 const uint32_t k_addr = smem_u32(sm + C::OFF_K + s * C::K_BYTES);
                 const uint32_t v_addr = smem_u32(sm + C::OFF_V + s * C::V_BYTES);
                 if (!wait1(sh, &bar[B_KV_FULL + s], (c >> 1) & 1, kWhereMmaKvFull)) break;
-                if (!wait1(sh, &bar[B_Q_FULL + qs], (c / C::QST) & 1, kWhereMmaQFull)) break;
+                if (!wait1(sh, &bar[B_Q_FULL + s], (c >> 1) & 1, kWhereMmaQFull)) break;
                 if (c >= 1 && !wait1(sh, &bar[B_S_EMPTY], (c - 1) & 1, kWhereMmaSEmpty)) break;
-                if (C::BIG && c >= 1 && !wait1(sh, &bar[B_H_EMPTY], (c - 1) & 1, kWhereMmaHEmpty)) break;
+                if (c >= 1 && prev_exact && !wait1(sh, &bar[B_H_EMPTY], (c - 1) & 1, kWhereMmaHEmpty)) break;
                 tc_fence_after();
                 // S = Q K^T
 #pragma unroll
@@ -286,39 +375,60 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 issued = true;
                 tc_commit(&bar[B_S_FULL]);
-                if (!wait1(sh, &bar[B_CONV], c & 1, kWhereMmaConv)) break;
+                if (!wait1(sh, &bar[B_G_FULL + slot], (c / kNG) & 1, kWhereMmaGate)) break;
+                const bool exact = gring[slot * C::G_FLOATS + kGScal + kSExact] != 0.f;
+                if (!wait1(sh, &bar[B_CONV0], c & 1, kWhereMmaConv)) break;
                 if (!wait1(sh, &bar[B_OPS], c & 1, kWhereMmaOps)) break;
-                if (!C::BIG && c >= 1 && !wait1(sh, &bar[B_H_EMPTY], (c - 1) & 1, kWhereMmaHEmpty)) break;
+                if (!exact && !wait1(sh, &bar[B_VT], c & 1, kWhereMmaVt)) break;
+                if (c >= 1 && !prev_exact && !wait1(sh, &bar[B_H_EMPTY], (c - 1) & 1, kWhereMmaHEmpty)) break;
                 tc_fence_after();
-                // H_inter = C_hi Q^T + C_lo Q^T
+                // H = C_hi Q^T + C_lo Q^T
 #pragma unroll
                 for (int ks = 0; ks < DQK / 16; ++ks) {
                     const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_f16_ts(tm + C::TM_HI, tm + C::TM_CHI + 8 * ks, smem_desc_sw128(q_addr + off, 16, 1024),
+                    mma_f16_ts(tm + C::TM_H, tm + C::TM_CHI + 8 * ks, smem_desc_sw128(q_addr + off, 16, 1024),
                                idR, ks > 0);
                 }
+                if (C::BIG) {
+                    for (int hf = 0; hf < 2; ++hf) {
+                        if (hf == 1) {
+                            tc_commit(&bar[B_CLO_FREE]);
+                            if (!wait1(sh, &bar[B_CONV1], c & 1, kWhereMmaClo)) goto mma_done;
+                            tc_fence_after();
+                        }
 #pragma unroll
-                for (int ks = 0; ks < DQK / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    if (C::BIG)
-                        mma_f16_ss(tm + C::TM_HI, smem_desc_sw128(clo_addr + (ks >> 2) * 16384 + (ks & 3) * 32, 16, 1024),
-                                   smem_desc_sw128(q_addr + off, 16, 1024), idR, 1);
-                    else
-                        mma_f16_ts(tm + C::TM_HI, tm + C::TM_CLO + 8 * ks, smem_desc_sw128(q_addr + off, 16, 1024),
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const int ks = 8 * hf + kk;
+                            const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
+                            mma_f16_ss(tm + C::TM_H,
+                                       smem_desc_sw128(clo_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                       smem_desc_sw128(q_addr + off, 16, 1024), idR, 1);
+                        }
+                    }
+                } else {
+#pragma unroll
+                    for (int ks = 0; ks < DQK / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        mma_f16_ts(tm + C::TM_H, tm + C::TM_CLO + 8 * ks, smem_desc_sw128(q_addr + off, 16, 1024),
                                    idR, 1);
+                    }
                 }
-                // H_intra = V^T P_hi^T + V^T P_lo^T
+                // intra part: fast chunks accumulate (w V)^T (mask S)^T onto H; exact
+                // chunks put V^T P^T into the S columns
 #pragma unroll
                 for (int part = 0; part < 2; ++part)
 #pragma unroll
                     for (int ks = 0; ks < kL / 16; ++ks)
-                        mma_f16_ss(tm + C::TM_HA, smem_desc_sw128(v_addr + ks * 2048, 8192, 1024),
+                        mma_f16_ss(exact ? tm + C::TM_S : tm + C::TM_H,
+                                   smem_desc_sw128(v_addr + ks * 2048, 8192, 1024),
                                    smem_desc_sw128(p_addr + part * 8192 + ks * 32, 16, 1024), idPV,
-                                   (part | ks) != 0);
+                                   exact ? (uint32_t)((part | ks) != 0) : 1u);
                 tc_commit(&bar[B_H_FULL]);
-                tc_commit(&bar[B_Q_EMPTY + qs]);
-                if (!wait1(sh, &bar[B_UPD_READY], c & 1, kWhereMmaUpd)) break;
-                tc_fence_after();
+                tc_commit(&bar[B_Q_EMPTY + s]);
+                if (exact) {
+                    if (!wait1(sh, &bar[B_VT], c & 1, kWhereMmaVt)) break;
+                    tc_fence_after();
+                }
                 // C_acc += (w V)^T K
 #pragma unroll
                 for (int ks = 0; ks < kL / 16; ++ks)
@@ -326,7 +436,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                                smem_desc_sw128(k_addr + ks * 2048, 8192, 1024), idU, 1);
                 tc_commit(&bar[B_UPD_DONE]);
                 tc_commit(&bar[B_KV_EMPTY + s]);
+                prev_exact = exact;
             }
+        mma_done:
             if (issued) {   // drain: all issued MMAs complete before tensor memory is freed
                 tc_commit(&bar[B_DRAIN]);
                 drain_wait(&bar[B_DRAIN], 0);
@@ -345,8 +457,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const double ia = ta < len ? (double)ig[t0 + ta] : -INFINITY, fa = ta < len ? (double)fg[t0 + ta] : 0.0;
             const double ib = tb < len ? (double)ig[t0 + tb] : -INFINITY, fb = tb < len ? (double)fg[t0 + tb] : 0.0;
             // inclusive prefix sum of f over the chunk
-            const double pair = fa + fb;
-            double incl = pair;
+            double incl = fa + fb;
 #pragma unroll
             for (int o = 1; o < 32; o <<= 1) {
                 const double y = __shfl_up_sync(0xffffffffu, incl, o);
@@ -367,26 +478,32 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (lane == 0) before = -INFINITY;
             const double mua = fmax(fmax(m, before), ua), mub = fmax(mua, ub);
             const double muL = __shfl_sync(0xffffffffu, mub, 31);
+            const double mu0 = __shfl_sync(0xffffffffu, mua, 0);
             const double FL = __shfl_sync(0xffffffffu, Fb, 31);
-            const bool rescale = muL - b > kRescale;
-            const double bnew = rescale ? muL : b;
+            const bool exact = muL - mu0 > kGrowth;
+            const double r = exact ? muL : (muL - b <= kRescale ? b : muL - kRescale);
             float *g = gring + slot * C::G_FLOATS;
             split_double(ua * kLog2e, g[kGUh + ta], g[kGUl + ta]);
             split_double(ub * kLog2e, g[kGUh + tb], g[kGUl + tb]);
             split_double(mua * kLog2e, g[kGMh + ta], g[kGMl + ta]);
             split_double(mub * kLog2e, g[kGMh + tb], g[kGMl + tb]);
-            g[kGA + ta] = p.scale * expf((float)(b - mua));
-            g[kGA + tb] = p.scale * expf((float)(b - mub));
-            g[kGW + ta] = expf((float)(ua - bnew));
-            g[kGW + tb] = expf((float)(ub - bnew));
+            const double aref = exact ? b : r;   // reference of the H coefficient
+            g[kGAH + ta] = p.scale * expf((float)(aref - mua));
+            g[kGAH + tb] = p.scale * expf((float)(aref - mub));
+            g[kGAN + ta] = p.scale * expf((float)(b - mua));
+            g[kGAN + tb] = p.scale * expf((float)(b - mub));
+            g[kGW + ta] = expf((float)(ua - r));
+            g[kGW + tb] = expf((float)(ub - r));
             g[kGLower + ta] = expf((float)(-(Fa + mua)));
             g[kGLower + tb] = expf((float)(-(Fb + mub)));
-            const float rho = expf((float)(b - bnew));
+            const float rho = expf((float)(b - r));
+            const bool rescale = r != b;
             m = FL + muL;
-            b = bnew + FL;
+            b = r + FL;
             if (lane == 0) {
                 g[kGScal + kSRho] = rho;
                 g[kGScal + kSRescale] = rescale ? 1.f : 0.f;
+                g[kGScal + kSExact] = exact ? 1.f : 0.f;
                 g[kGScal + kSMEnd] = (float)m;
                 g[kGScal + kSGsc] = expf((float)(b - m));   // final-state gauge factor e^{b-m}
             }
@@ -418,6 +535,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int i = 0; i < NPL; ++i) nacc[i] *= rho;
             const uint8_t *Ks = sm + C::OFF_K + s * C::K_BYTES;
             const uint32_t box = j0 >> 6, chunk = (j0 & 63) >> 3, within = (j0 & 7) * 2;
+#pragma unroll 4
             for (int t = 0; t < kL; ++t) {
                 const float w = g[kGW + t];
                 const uint8_t *src = Ks + box * 8192 + sw128_offset(t, chunk) + within;
@@ -453,16 +571,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < NPL; ++i) p.n1[(size_t)bh * DQK + j0 + i] = nacc[i] * gsc;
         }
-    } else {
-        // ===================== state split, P, epilogue (warps 4-7) =====================
-        const int ct = tid - 128;            // 0..127: TMEM lane / C row of this block
+    } else if (warp < 8) {
+        // ===================== state group (warps 4-7) =====================
+        const int st = tid - 128;            // 0..127: TMEM lane / value row of this block
         const int wq = warp - 4;             // TMEM lane quarter
         const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
-        const int v = v0 + ct;
+        const int v = v0 + st;
         float *hout = p.h + (size_t)bh * T * p.dv + v;
         uint8_t *clo_s = sm + C::OFF_CLO;
-        // initial state into tensor memory: C_acc = C0 (b = m = m0) or zero
-        {
+        {   // initial state: C_acc = C0 (gauge b = m = m0) or zero
             float r[32];
             const float *src = p.C0 ? p.C0 + ((size_t)bh * p.dv + v) * DQK : nullptr;
 #pragma unroll 1
@@ -473,124 +590,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tmem_wait_st();
         }
+        named_barrier(3, 256);   // C_acc is initialised before either group splits it
         bool alive = true;
         float m_end = p.m0 ? p.m0[bh] : 0.f, gsc = 1.f;
-        const int trow = ct >> 1, half = ct & 1;     // nq pass: row and half of d_qk
         for (int c = 0; c < NC; ++c) {
-            const int slot = c % kNG, s = c & 1, qs = c % C::QST;
+            const int slot = c % kNG, s = c & 1, sb = c & 1;
             const float *g = gring + slot * C::G_FLOATS;
-            // --- split the state at chunk start into C_hi + C_lo (bf16 pair)
-            if (c >= 1) alive = alive && waitw(sh, &bar[B_UPD_DONE], (c - 1) & 1, kWhereCwUpd);
+            if (c >= 1) alive = alive && waitw(sh, &bar[B_UPD_DONE], (c - 1) & 1, kWhereStUpd);
+            alive = alive && waitw(sh, &bar[B_G_FULL + slot], (c / kNG) & 1, kWhereStGate);
+            const bool exact = alive && g[kGScal + kSExact] != 0.f;
+            // --- lower half of the state split (C_lo of it: TMEM, or the shared tile)
             if (alive) {
                 tc_fence_after();
-                float r[32];
+                const bool mv = !exact && g[kGScal + kSRescale] != 0.f;
+                const float rho = g[kGScal + kSRho];
 #pragma unroll 1
-                for (int i = 0; i < DQK / 32; ++i) {
-                    tmem_ld32(tm + lane_base + C::TM_C + 32 * i, r);
-                    tmem_wait_ld();
-                    uint32_t hi[16], lo[16];
-#pragma unroll
-                    for (int x = 0; x < 16; ++x) {
-                        hi[x] = pack_bf16x2(r[2 * x], r[2 * x + 1]);
-                        lo[x] = pack_bf16x2(r[2 * x] - bf_lo(hi[x]), r[2 * x + 1] - bf_hi(hi[x]));
-                    }
-                    tmem_st16(tm + lane_base + C::TM_CHI + 16 * i, hi);
-                    if (C::BIG) {
-                        // K-major 128B-swizzled [128 rows][d_qk] bf16 tile, row ct
-#pragma unroll
-                        for (int q4 = 0; q4 < 4; ++q4) {
-                            const int j = 32 * i + 8 * q4;
-                            *reinterpret_cast<uint4 *>(clo_s + (j >> 6) * 16384 + sw128_offset(ct, (j & 63) >> 3)) =
-                                make_uint4(lo[4 * q4], lo[4 * q4 + 1], lo[4 * q4 + 2], lo[4 * q4 + 3]);
-                        }
-                    } else {
-                        tmem_st16(tm + lane_base + C::TM_CLO + 16 * i, lo);
-                    }
-                }
+                for (int i = 0; i < DQK / 64; ++i)
+                    split_state_block<C>(tm, lane_base, i, mv, rho, C::BIG ? 1 : 0, clo_s, st, 32 * i);
                 tmem_wait_st();
                 if (C::BIG) fence_proxy_async_smem();
                 tc_fence_before();
             }
             named_barrier(1, 128);
-            if (ct == 0 && alive) mbar_arrive(&bar[B_CONV]);
-            // --- nq_t = a_t (n_acc . q_t) in fp32
-            alive = alive && waitw(sh, &bar[B_G_FULL + slot], (c / kNG) & 1, kWhereCwGate);
-            alive = alive && waitw(sh, &bar[B_Q_FULL + qs], (c / C::QST) & 1, kWhereCwQ);
-            alive = alive && waitw(sh, &bar[B_N_READY + (c & 1)], (c >> 1) & 1, kWhereCwN);
-            if (alive) {
-                const uint8_t *Qs = sm + C::OFF_Q + qs * C::Q_BYTES;
-                const float *nn = nbuf + (c & 1) * DQK;
-                float nq = 0.f;
-#pragma unroll 4
-                for (int gi = 0; gi < DQK / 16; ++gi) {
-                    const int j = half * (DQK / 2) + 8 * gi;
-                    const uint4 u = *reinterpret_cast<const uint4 *>(Qs + (j >> 6) * 8192 + sw128_offset(trow, (j & 63) >> 3));
-                    float x[8];
-                    unpack_bf16x8(u, x);
-                    const float4 n0 = *reinterpret_cast<const float4 *>(nn + j);
-                    const float4 n1 = *reinterpret_cast<const float4 *>(nn + j + 4);
-                    nq = fmaf(x[0], n0.x, nq); nq = fmaf(x[1], n0.y, nq);
-                    nq = fmaf(x[2], n0.z, nq); nq = fmaf(x[3], n0.w, nq);
-                    nq = fmaf(x[4], n1.x, nq); nq = fmaf(x[5], n1.y, nq);
-                    nq = fmaf(x[6], n1.z, nq); nq = fmaf(x[7], n1.w, nq);
-                }
-                nq += __shfl_xor_sync(0xffffffffu, nq, 1);
-                if (half == 0) nq_s[trow] = g[kGA + trow] * nq;
+            if (st == 0 && alive) mbar_arrive(&bar[B_CONV0]);
+            // --- denominators, once the token group has published n.q and the row sums
+            alive = alive && waitw(sh, &bar[B_OPS], c & 1, kWhereStOps);
+            if (alive && st < kL) {
+                const float inv = 1.f / fmaxf(fabsf(nq_s[sb * kL + st] + rs_s[sb * kL + st]), g[kGLower + st]);
+                inv_s[sb * kL + st] = inv;
+                coef_s[sb * kL + st] = g[kGAH + st] * inv;
             }
             named_barrier(1, 128);
-            if (ct == 0 && alive) {
-                mbar_arrive(&bar[B_Q_EMPTY + qs]);
-                mbar_arrive(&bar[B_N_FREE + (c & 1)]);
-            }
-            // --- P = scale S e^{u_s - mu_t} on s <= t as a bf16 hi/lo pair
-            alive = alive && waitw(sh, &bar[B_S_FULL], c & 1, kWhereCwS);
+            alive = alive && waitw(sh, &bar[B_H_FULL], c & 1, kWhereStH);
             if (alive) {
                 tc_fence_after();
-                float r0[32], r1[32];
-                tmem_ld32(tm + lane_base + C::TM_S, r0);
-                tmem_ld32(tm + lane_base + C::TM_S + 32, r1);
-                tmem_wait_ld();
-                if (lane < 16) {
-                    const int t = 16 * wq + lane;
-                    const float mh = g[kGMh + t], ml = g[kGMl + t];
-                    float rs = 0.f;
-#pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        uint32_t hi[4], lo[4];
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int s0 = 8 * ch + 2 * i;
-                            const float sa = (s0 < 32) ? r0[s0] : r1[s0 - 32];
-                            const float sb = (s0 + 1 < 32) ? r0[s0 + 1] : r1[s0 - 31];
-                            const float ea = (g[kGUh + s0] - mh) + (g[kGUl + s0] - ml);
-                            const float eb = (g[kGUh + s0 + 1] - mh) + (g[kGUl + s0 + 1] - ml);
-                            const float pa = (s0 <= t) ? p.scale * sa * exp2f(ea) : 0.f;
-                            const float pb = (s0 + 1 <= t) ? p.scale * sb * exp2f(eb) : 0.f;
-                            hi[i] = pack_bf16x2(pa, pb);
-                            lo[i] = pack_bf16x2(pa - bf_lo(hi[i]), pb - bf_hi(hi[i]));
-                            rs += pa + pb;
-                        }
-                        *reinterpret_cast<uint4 *>(Ps + sw128_offset(t, ch)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                        *reinterpret_cast<uint4 *>(Ps + 8192 + sw128_offset(t, ch)) =
-                            make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                    }
-                    rs_s[t] = rs;
-                }
-                tc_fence_before();
-                fence_proxy_async_smem();
-            }
-            named_barrier(1, 128);
-            if (ct == 0 && alive) {
-                mbar_arrive(&bar[B_S_EMPTY]);
-                mbar_arrive(&bar[B_OPS]);
-            }
-            if (alive && ct < kL)
-                inv_s[ct] = 1.f / fmaxf(fabsf(nq_s[ct] + rs_s[ct]), g[kGLower + ct]);
-            // --- after the readout: gauge move of C_acc, then V <- w V in place
-            alive = alive && waitw(sh, &bar[B_H_FULL], c & 1, kWhereCwH);
-            if (alive) {
-                tc_fence_after();
-                if (g[kGScal + kSRescale] != 0.f) {   // C_acc *= e^{b - b'}
+                if (exact) {   // exact chunk: gauge move to r = mu_L, then V <- w V
                     const float rho = g[kGScal + kSRho];
                     float r[32];
 #pragma unroll 1
@@ -602,38 +636,42 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tmem_st32(tm + lane_base + C::TM_C + 32 * i, r);
                     }
                     tmem_wait_st();
+                    scale_v_rows(sm + C::OFF_V + s * C::V_BYTES, g + kGW, st);
+                    fence_proxy_async_smem();
+                    tc_fence_before();
                 }
-                uint8_t *Vs = sm + C::OFF_V + s * C::V_BYTES;
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                    const int e = ct + 128 * i;              // 16-byte chunk index in the stage
-                    const float w = g[kGW + ((e & 511) >> 3)];   // rows are tokens
-                    uint4 *ptr = reinterpret_cast<uint4 *>(Vs + 16 * e);
-                    float x[8];
-                    unpack_bf16x8(*ptr, x);
-                    *ptr = make_uint4(pack_bf16x2(w * x[0], w * x[1]), pack_bf16x2(w * x[2], w * x[3]),
-                                      pack_bf16x2(w * x[4], w * x[5]), pack_bf16x2(w * x[6], w * x[7]));
-                }
-                fence_proxy_async_smem();
-                tc_fence_before();
             }
-            named_barrier(1, 128);
-            if (ct == 0 && alive) mbar_arrive(&bar[B_UPD_READY]);
-            // --- epilogue: h~[t][v] = (a_t H_inter[v][t] + H_intra[v][t]) / den_t
+            named_barrier(1, 128);   // unconditional: every warp of the group takes every barrier
+            if (st == 0 && alive && exact) mbar_arrive(&bar[B_VT]);
+            // --- epilogue: h~[t][v] = (AH_t H[v][t] (+ intra[v][t])) / den_t
             if (alive) {
                 const int len = min(kL, T - kL * c);
                 float *hc = hout + (size_t)kL * c * p.dv;
-#pragma unroll
+#pragma unroll 1
                 for (int hh = 0; hh < 2; ++hh) {
-                    float ri[32], ra[32];
-                    tmem_ld32(tm + lane_base + C::TM_HI + 32 * hh, ri);
-                    tmem_ld32(tm + lane_base + C::TM_HA + 32 * hh, ra);
+                    float rh[32], cf[32];
+                    tmem_ld32(tm + lane_base + C::TM_H + 32 * hh, rh);
+                    load32(coef_s + sb * kL + 32 * hh, cf);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int x = 0; x < 32; ++x) {
-                        const int t = 32 * hh + x;
-                        const float hv = fmaf(g[kGA + t], ri[x], ra[x]) * inv_s[t];
-                        if (t < len) hc[(size_t)t * p.dv] = hv;
+                    for (int x = 0; x < 32; ++x) rh[x] *= cf[x];
+                    if (exact) {
+                        float ra[32];
+                        tmem_ld32(tm + lane_base + C::TM_S + 32 * hh, ra);
+                        load32(inv_s + sb * kL + 32 * hh, cf);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) rh[x] = fmaf(ra[x], cf[x], rh[x]);
+                    }
+                    float *hrow = hc + (size_t)32 * hh * p.dv;
+                    const int n = min(32, len - 32 * hh);
+                    if (n == 32) {
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) hrow[(size_t)x * p.dv] = rh[x];
+                    } else {
+#pragma unroll
+                        for (int x = 0; x < 32; ++x)
+                            if (x < n) hrow[(size_t)x * p.dv] = rh[x];
                     }
                 }
                 m_end = g[kGScal + kSMEnd];
@@ -641,13 +679,13 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_before();
             }
             named_barrier(1, 128);
-            if (ct == 0 && alive) {
+            if (st == 0 && alive) {
                 mbar_arrive(&bar[B_H_EMPTY]);
                 mbar_arrive(&bar[B_G_EMPTY + slot]);
             }
         }
         // final state: C~ = e^{b - m} C_acc
-        alive = alive && waitw(sh, &bar[B_UPD_DONE], (NC - 1) & 1, kWhereCwFinal);
+        alive = alive && waitw(sh, &bar[B_UPD_DONE], (NC - 1) & 1, kWhereStFinal);
         if (alive) {
             tc_fence_after();
             if (p.C1) {
@@ -663,9 +701,158 @@ __global__ void __launch_bounds__(kThreads, 1)
                             make_float4(r[x] * gsc, r[x + 1] * gsc, r[x + 2] * gsc, r[x + 3] * gsc);
                 }
             }
-            if (slice == 0 && ct == 0 && p.m1) p.m1[bh] = m_end;
+            if (slice == 0 && st == 0 && p.m1) p.m1[bh] = m_end;
         }
         tc_fence_before();
+    } else {
+        // ===================== token group (warps 8-11) =====================
+        const int tk = tid - 256;            // 0..127
+        const int wq = warp - 8;             // TMEM lane quarter
+        const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
+        const int trow = tk >> 1, half = tk & 1;     // n.q pass: token row, half of d_qk
+        uint8_t *clo_s = sm + C::OFF_CLO;
+        named_barrier(3, 256);   // C_acc is initialised before either group splits it
+        bool alive = true;
+        for (int c = 0; c < NC; ++c) {
+            const int slot = c % kNG, s = c & 1, sb = c & 1;
+            const float *g = gring + slot * C::G_FLOATS;
+            // the P tile, n.q / row-sum slots and the V stage of chunk c-2 are free
+            if (c >= 1) alive = alive && waitw(sh, &bar[B_H_FULL], (c - 1) & 1, kWhereTkH);
+            alive = alive && waitw(sh, &bar[B_G_FULL + slot], (c / kNG) & 1, kWhereTkGate);
+            const bool exact = alive && g[kGScal + kSExact] != 0.f;
+            // --- fast chunk: V <- w V in place, before the intra product
+            alive = alive && waitw(sh, &bar[B_KV_FULL + s], (c >> 1) & 1, kWhereTkKv);
+            if (alive && !exact) {
+                scale_v_rows(sm + C::OFF_V + s * C::V_BYTES, g + kGW, tk);
+                fence_proxy_async_smem();
+            }
+            named_barrier(2, 128);   // unconditional: every warp of the group takes every barrier
+            if (tk == 0 && alive && !exact) mbar_arrive(&bar[B_VT]);
+            // --- upper half of the state split (its C_lo waits for the shared tile when d_qk = 256)
+            if (c >= 1) alive = alive && waitw(sh, &bar[B_UPD_DONE], (c - 1) & 1, kWhereTkUpd);
+            if (alive) {
+                tc_fence_after();
+                const bool mv = !exact && g[kGScal + kSRescale] != 0.f;
+                const float rho = g[kGScal + kSRho];
+#pragma unroll 1
+                for (int i = DQK / 64; i < DQK / 32; ++i)
+                    split_state_block<C>(tm, lane_base, i, mv, rho, C::BIG ? 2 : 0, clo_s, tk, 0);
+                tmem_wait_st();
+                tc_fence_before();
+            }
+            named_barrier(2, 128);
+            if (tk == 0 && alive) mbar_arrive(&bar[B_CONV0]);
+            // --- n.q_t in fp32 (coefficient AN_t = scale e^{b - mu_t})
+            alive = alive && waitw(sh, &bar[B_Q_FULL + s], (c >> 1) & 1, kWhereTkQ);
+            alive = alive && waitw(sh, &bar[B_N_READY + (c & 1)], (c >> 1) & 1, kWhereTkN);
+            if (alive) {
+                const uint8_t *Qs = sm + C::OFF_Q + s * C::Q_BYTES;
+                const float *nn = nbuf + (c & 1) * DQK;
+                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                 make_float2(0.f, 0.f)};
+#pragma unroll 1
+                for (int g0 = 0; g0 < DQK / 16; g0 += 4) {
+                    uint4 u[4];
+                    float4 na[4], nb[4];
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        const int j = half * (DQK / 2) + 8 * (g0 + k4);
+                        u[k4] = *reinterpret_cast<const uint4 *>(Qs + (j >> 6) * 8192 + sw128_offset(trow, (j & 63) >> 3));
+                        na[k4] = *reinterpret_cast<const float4 *>(nn + j);
+                        nb[k4] = *reinterpret_cast<const float4 *>(nn + j + 4);
+                    }
+#pragma unroll
+                    for (int k4 = 0; k4 < 4; ++k4) {
+                        acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].x), make_float2(na[k4].x, na[k4].y), acc[k4]);
+                        acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].y), make_float2(na[k4].z, na[k4].w), acc[k4]);
+                        acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].z), make_float2(nb[k4].x, nb[k4].y), acc[k4]);
+                        acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].w), make_float2(nb[k4].z, nb[k4].w), acc[k4]);
+                    }
+                }
+                float nq = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+                nq += __shfl_xor_sync(0xffffffffu, nq, 1);
+                if (half == 0) nq_s[sb * kL + trow] = g[kGAN + trow] * nq;
+            }
+            named_barrier(2, 128);
+            if (tk == 0 && alive) {
+                mbar_arrive(&bar[B_Q_EMPTY + s]);
+                mbar_arrive(&bar[B_N_FREE + (c & 1)]);
+            }
+            // --- P from S: lanes l and l+16 share token row 16 wq + (l & 15)
+            alive = alive && waitw(sh, &bar[B_S_FULL], c & 1, kWhereTkS);
+            if (alive) {
+                tc_fence_after();
+                float r0[32], r1[32];
+                tmem_ld32(tm + lane_base + C::TM_S, r0);
+                tmem_ld32(tm + lane_base + C::TM_S + 32, r1);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 32; ++i) {
+                    const float up = __shfl_sync(0xffffffffu, r1[i], lane & 15);
+                    if (lane >= 16) r0[i] = up;
+                }
+                const int t = 16 * wq + (lane & 15);
+                const int s0 = 32 * (lane >> 4);
+                float rs = 0.f;
+                if (exact) {
+                    const float mh = g[kGMh + t], ml = g[kGMl + t];
+                    float uh[32], ul[32];
+                    load32(g + kGUh + s0, uh);
+                    load32(g + kGUl + s0, ul);
+#pragma unroll
+                    for (int i = 0; i < 32; ++i) {
+                        const int sidx = s0 + i;
+                        const float e = (uh[i] - mh) + (ul[i] - ml);
+                        r0[i] = (sidx <= t) ? p.scale * r0[i] * exp2f(e) : 0.f;
+                        rs += r0[i];
+                    }
+                } else {
+                    float ww[32];
+                    load32(g + kGW + s0, ww);
+                    float2 r2 = make_float2(0.f, 0.f);
+#pragma unroll
+                    for (int i = 0; i < 32; i += 2) {
+                        r0[i] = (s0 + i <= t) ? r0[i] : 0.f;
+                        r0[i + 1] = (s0 + i + 1 <= t) ? r0[i + 1] : 0.f;
+                        r2 = __ffma2_rn(make_float2(r0[i], r0[i + 1]), make_float2(ww[i], ww[i + 1]), r2);
+                    }
+                    rs = r2.x + r2.y;
+                }
+#pragma unroll
+                for (int ch = 0; ch < 4; ++ch) {
+                    uint32_t hi[4], lo[4];
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) split_bf16x2(r0[8 * ch + 2 * i], r0[8 * ch + 2 * i + 1], hi[i], lo[i]);
+                    const int chunk = 4 * (lane >> 4) + ch;
+                    *reinterpret_cast<uint4 *>(Ps + sw128_offset(t, chunk)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+                    *reinterpret_cast<uint4 *>(Ps + 8192 + sw128_offset(t, chunk)) =
+                        make_uint4(lo[0], lo[1], lo[2], lo[3]);
+                }
+                rs += __shfl_xor_sync(0xffffffffu, rs, 16);
+                if (lane < 16) rs_s[sb * kL + t] = exact ? rs : g[kGAH + t] * rs;
+                tc_fence_before();
+                fence_proxy_async_smem();
+            }
+            named_barrier(2, 128);
+            if (tk == 0 && alive) {
+                mbar_arrive(&bar[B_S_EMPTY]);
+                mbar_arrive(&bar[B_OPS]);
+                mbar_arrive(&bar[B_G_EMPTY + slot]);
+            }
+            if (C::BIG) {   // second half of C_lo once the MMA has consumed the first
+                alive = alive && waitw(sh, &bar[B_CLO_FREE], c & 1, kWhereTkClo);
+                if (alive) {
+                    tc_fence_after();
+#pragma unroll 1
+                    for (int i = DQK / 64; i < DQK / 32; ++i)
+                        split_state_block<C>(tm, lane_base, i, false, 1.f, 3, clo_s, tk, 32 * i - DQK / 2);
+                    fence_proxy_async_smem();
+                    tc_fence_before();
+                }
+                named_barrier(2, 128);
+                if (tk == 0 && alive) mbar_arrive(&bar[B_CONV1]);
+            }
+        }
     }
 
     __syncthreads();
