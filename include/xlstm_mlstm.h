@@ -142,6 +142,37 @@ XLSTM_API xlstm_status_t xlstm_mlstm_step(
     float *h_out, float *C_new, float *n_new, float *m_new,
     cudaStream_t stream);
 
+/*
+ * xlstm_mlstm_fwd_chunkwise without a caller workspace, for callers that cannot
+ * allocate device memory: a plug-in inside a host framework that owns every
+ * device allocation and offers no allocator, or code on a latency-critical path
+ * where cudaMalloc (which may synchronise the device and may fail) is not
+ * allowed.  (The xLSTM pages have no counterpart to this call; it is a library
+ * convenience.)
+ *
+ * Same arguments, rules and results as xlstm_mlstm_fwd_chunkwise, minus the
+ * workspace.  The scratch is a fixed 4096-byte array in the library's own
+ * device memory, held on every GPU that loads the library until the process
+ * exits; a desc whose xlstm_mlstm_workspace_size exceeds 4096 bytes is refused
+ * with XLSTM_ERR_WORKSPACE.  The call allocates nothing and frees nothing.
+ *   - The first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress, with that device current); make that first call
+ *     before capturing any stream.
+ *   - All calls share the one array: calls that overlap on the device (other
+ *     streams, other host threads) race on it.  Each call clears the part that
+ *     must start at zero (the status block) on its stream before its kernel.
+ *   - The device status block lives in that array and is not readable through
+ *     this API; use xlstm_mlstm_fwd_chunkwise with a workspace when the status
+ *     of the device-side waits is needed.
+ */
+XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise_noalloc(
+    const xlstm_mlstm_desc_t *desc,
+    const void *q, const void *k, const void *v,
+    const float *i_pre, const float *f_pre,
+    const float *C_in, const float *n_in, const float *m_in,
+    float *h_out, float *C_out, float *n_out, float *m_out,
+    cudaStream_t stream);
+
 /* Workspace bytes xlstm_mlstm_fwd_chunkwise needs for desc (>= 256), or 0 for
  * a NULL desc. */
 XLSTM_API size_t xlstm_mlstm_workspace_size(const xlstm_mlstm_desc_t *desc);

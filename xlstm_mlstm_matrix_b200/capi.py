@@ -20,7 +20,8 @@ XLSTM_F32, XLSTM_BF16 = 0, 1
 
 EXPORTED = ("xlstm_mlstm_fwd_chunkwise", "xlstm_mlstm_fwd_recurrent", "xlstm_mlstm_step",
             "xlstm_mlstm_workspace_size", "xlstm_mlstm_workspace_status", "xlstm_status_string",
-            "xlstm_mlstm_version", "xlstm_mlstm_chunkwise_kernel", "xlstm_mlstm_test_timeout_next")
+            "xlstm_mlstm_version", "xlstm_mlstm_chunkwise_kernel", "xlstm_mlstm_test_timeout_next",
+            "xlstm_mlstm_fwd_chunkwise_noalloc")
 
 
 class xlstm_mlstm_desc_t(ctypes.Structure):
@@ -52,6 +53,8 @@ def load(path: str = LIB_PATH):
     for name in ("xlstm_mlstm_fwd_chunkwise", "xlstm_mlstm_fwd_recurrent"):
         getattr(lib, name).argtypes = seq
         getattr(lib, name).restype = st
+    lib.xlstm_mlstm_fwd_chunkwise_noalloc.argtypes = [dp] + [vp] * 12 + [vp]
+    lib.xlstm_mlstm_fwd_chunkwise_noalloc.restype = st
     lib.xlstm_mlstm_step.argtypes = [dp] + [vp] * 12 + [vp]
     lib.xlstm_mlstm_step.restype = st
     lib.xlstm_mlstm_workspace_size.argtypes = [dp]
@@ -100,6 +103,15 @@ def xlstm_mlstm_fwd_chunkwise(desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in, h_o
         ctypes.byref(desc), _p(q), _p(k), _p(v), _p(i_pre), _p(f_pre), _p(C_in), _p(n_in),
         _p(m_in), _p(h_out), _p(C_out), _p(n_out), _p(m_out), _p(workspace), workspace_bytes,
         _s(stream))
+
+
+def xlstm_mlstm_fwd_chunkwise_noalloc(desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in, h_out, C_out,
+                                      n_out, m_out, stream=None) -> int:
+    """Chunkwise forward using the library's fixed scratch array instead of a
+    caller workspace (for callers that cannot allocate device memory)."""
+    return load().xlstm_mlstm_fwd_chunkwise_noalloc(
+        ctypes.byref(desc), _p(q), _p(k), _p(v), _p(i_pre), _p(f_pre), _p(C_in), _p(n_in),
+        _p(m_in), _p(h_out), _p(C_out), _p(n_out), _p(m_out), _s(stream))
 
 
 def xlstm_mlstm_fwd_recurrent(desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in, h_out, C_out,
