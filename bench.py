@@ -6,6 +6,12 @@ fp32 gates, zero initial state, fp32 h~ and final state), synthetic seeded
 inputs.  One step = one xlstm_mlstm_fwd_chunkwise call over the whole batch.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload layer_7b|long_context|many_short|decode]
+
+The default workload is the 7B-like layer.  --workload picks another of the
+synthetic workloads: a sequence workload runs one chunkwise call per step; the
+decode workload (B=128, H=8, d_qk=256, d_v=512, state resident in HBM) runs one
+xlstm_mlstm_step call per step and counts B tokens per step.
 
 value      tokens/s (B*T positions per step) with inputs resident in HBM,
            timed with CUDA events on the launch stream, max over ranks;
@@ -34,7 +40,7 @@ import numpy as np
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-WORKLOAD = "layer_7b"
+DEFAULT_WORKLOAD = "layer_7b"
 METRIC = "mLSTM fwd tokens/s & TFLOP/s on 1 B200; % of tensor/HBM roofline"
 UNIT = "tokens/s"
 
@@ -48,12 +54,23 @@ def peaks():
 
 
 def algorithmic(w, L=64):
-    """Bytes and flops one forward moves/does (counting convention of the design notes)."""
-    N = w.B * w.H * w.T
+    """Bytes and flops of one step (counting convention of the design notes).
+
+    Sequence workloads: one forward over B*H*T head-tokens; inputs, h~ and the
+    final state (plus the initial state when one is read).  Decode: one step
+    over B*H heads; the state is read and written once, plus the step's vectors.
+    """
     e = 2 if w.dtype == "bf16" else 4
-    bytes_ = N * ((2 * w.d_qk + w.d_v) * e + 8 + 4 * w.d_v) + w.B * w.H * (w.d_qk * w.d_v + w.d_qk + 1) * 4
+    state = w.d_qk * w.d_v + w.d_qk + 1
+    if w.steps:
+        BH = w.B * w.H
+        bytes_ = BH * ((2 * w.d_qk + w.d_v) * e + 8 + 4 * w.d_v + 2 * 4 * state)
+        flops = BH * (5 * w.d_qk * w.d_v + 4 * w.d_qk)
+        return bytes_, flops
+    N = w.B * w.H * w.T
+    bytes_ = N * ((2 * w.d_qk + w.d_v) * e + 8 + 4 * w.d_v) + w.B * w.H * state * 4
     if w.state != "zero":
-        bytes_ += w.B * w.H * (w.d_qk * w.d_v + w.d_qk + 1) * 4
+        bytes_ += w.B * w.H * state * 4
     flops = N * (4 * w.d_qk * w.d_v + L * (w.d_qk + w.d_v))
     return bytes_, flops
 
@@ -116,14 +133,14 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def traffic_for(kernel_src_sha: str):
+def traffic_for(kernel_src_sha: str, workload: str):
     """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source; else None."""
+    on the current kernel source for this workload; else None."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
-    d = json.load(open(path))
-    if d.get("source_sha") != kernel_src_sha or d.get("workload") != WORKLOAD:
+    d = json.load(open(path)).get(workload)
+    if not d or d.get("source_sha") != kernel_src_sha:
         return None
     return d.get("traffic_bytes_per_launch")
 
@@ -137,13 +154,47 @@ def kernel_source_sha():
     return h.hexdigest()[:16]
 
 
-def cpu_baseline(inp, budget_s=12.0):
-    """Time the float64 oracle on a bounded sample: whole sequences of a few
-    heads, all host threads.  Returns tokens/s in the workload's units."""
+def tokens_per_step(w):
+    return w.B if w.steps else w.B * w.T
+
+
+def config_of(w, extra=None):
+    c = {"workload": w.name, "B": w.B, "H": w.H, "T": w.T if not w.steps else 1,
+         "d_qk": w.d_qk, "d_v": w.d_v}
+    if w.steps:
+        c["decode_steps"] = w.steps
+    c.update(extra or {})
+    return c
+
+
+def cpu_baseline(w, inp, budget_s=12.0):
+    """Time the float64 oracle on a bounded sample of the workload, all host
+    threads.  Returns the rate in the workload's tokens/s."""
     import oracle
-    w = inp["workload"]
     threads = oracle.default_threads()
-    sel = lambda x, hs: None if x is None else x.reshape((w.B * w.H,) + x.shape[2:])[hs][None]
+    flat = lambda x: None if x is None else x.reshape((w.B * w.H,) + x.shape[2:])
+    if w.steps:
+        # decode: every (b, h) of a sample, a few steps each, state carried
+        rng, C0, n0, m0 = inp["state"]
+        nheads = min(w.B * w.H, max(threads * 4, 1))
+        sel = lambda x: flat(x)[:nheads][None]
+        C, n, m = sel(C0), sel(n0), sel(m0)
+        t0 = time.perf_counter()
+        nsteps = 0
+        while True:
+            st = inp["steps"][nsteps % len(inp["steps"])]
+            _, C, n, m = oracle.step(*(sel(st[k]) for k in ("q", "k", "v", "i_pre", "f_pre")),
+                                     C, n, m, qk_scale=inp["qk_scale"], threads=threads)
+            nsteps += 1
+            dt = time.perf_counter() - t0
+            if dt >= budget_s or nsteps >= w.steps:
+                break
+        tokens = nsteps * nheads / w.H
+        return {"value": tokens / dt, "unit": UNIT, "cores": min(threads, nheads), "kind": "oracle",
+                "sample": f"{nsteps} decode steps of {nheads} of {w.B * w.H} (batch, head) pairs, "
+                          f"float64, {min(threads, nheads)} threads; tokens = head-steps / H",
+                "seconds": dt}
+    sel = lambda x, hs: None if x is None else flat(x)[hs][None]
     # probe with a short prefix of one head to size the sample
     Tp = min(w.T, 256)
     t0 = time.perf_counter()
@@ -151,10 +202,9 @@ def cpu_baseline(inp, budget_s=12.0):
                    qk_scale=inp["qk_scale"], threads=1)
     per_head_token = (time.perf_counter() - t0) / Tp
     nheads = int(max(1, min(w.B * w.H, threads * budget_s / max(per_head_token * w.T, 1e-9))))
-    nheads = max(1, min(nheads, threads * 2, w.B * w.H))
     hs = list(range(nheads))
     t0 = time.perf_counter()
-    oracle.forward(*(sel(inp[n], hs) for n in ("q", "k", "v", "i_pre", "f_pre")),
+    oracle.forward(*(sel(inp[n], hs) for n in ("q", "k", "v", "i_pre", "f_pre", "C0", "n0", "m0")),
                    qk_scale=inp["qk_scale"], threads=threads)
     dt = time.perf_counter() - t0
     tokens = nheads * w.T / w.H          # head-tokens / heads per token
@@ -164,30 +214,172 @@ def cpu_baseline(inp, budget_s=12.0):
             "seconds": dt}
 
 
+def workload_for_rank(name, rank, B=0, H=0, T=0):
+    """The workload one rank runs: every rank runs a full replica with its own
+    seed (heads are independent, so ranks share nothing on the data path)."""
+    from xlstm_mlstm_matrix_b200 import inputs
+    base = inputs.WORKLOADS[name]
+    w = base.replace(seed=base.seed + 1000 * rank)
+    if B or H or T:   # a smaller case of the same layer (profiling captures)
+        w = w.replace(B=B or w.B, H=H or w.H, T=T or w.T)
+    return w
+
+
+def max_over_ranks(x, dist=None, device=None):
+    """The slowest rank's value (a float), identical on every rank."""
+    if dist is None:
+        return x
+    import torch
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(tokens_per_rank, world, ms_max):
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time."""
+    return world * tokens_per_rank / (ms_max * 1e-3)
+
+
+def make_inputs(w, n_decode_steps=None):
+    from xlstm_mlstm_matrix_b200 import inputs
+    if not w.steps:
+        return inputs.make_sequence(w)
+    rng, C0, n0, m0 = inputs.decode_state(w)
+    steps = list(inputs.decode_steps(w, rng, n_decode_steps))
+    return {"state": (rng, C0, n0, m0), "steps": steps, "qk_scale": float(1.0 / np.sqrt(w.d_qk)),
+            "workload": w}
+
+
 def run_reference(args, rank, world):
     """--impl reference: the float64 oracle on host cores, same metric/workload."""
     from xlstm_mlstm_matrix_b200 import inputs
     if rank != 0:
         return
-    w = inputs.WORKLOADS[WORKLOAD]
-    inp = inputs.make_sequence(w)
+    w = inputs.WORKLOADS[args.workload]
+    inp = make_inputs(w, n_decode_steps=32)
     # each step is a bounded sample so that the whole run stays within minutes
     budget = max(2.0, min(args.ref_budget, 150.0 / max(1, args.steps)))
     vals = []
     cb = None
     for _ in range(max(1, args.steps)):
-        cb = cpu_baseline(inp, budget_s=budget)
+        cb = cpu_baseline(w, inp, budget_s=budget)
         vals.append(cb["value"])
     value = statistics.median(vals)
     cb["value"] = value
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
-            "warmup": args.warmup, "ms_per_step": 1e3 * w.tokens / value,
+            "warmup": args.warmup, "ms_per_step": 1e3 * tokens_per_step(w) / value,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "impl": "reference",
-            "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "T": w.T, "d_qk": w.d_qk, "d_v": w.d_v},
+            "data": "synthetic", "impl": "reference", "config": config_of(w),
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
+
+
+class _Sequence:
+    """One chunkwise forward over the whole batch per step."""
+
+    def __init__(self, w, inp, dev, stream):
+        import torch
+        from xlstm_mlstm_matrix_b200 import capi
+        self.w, self.inp = w, inp
+        bf = w.dtype == "bf16"
+        dev_t = lambda x, b: None if x is None else (
+            torch.from_numpy(x).to(dev).to(torch.bfloat16) if b else torch.from_numpy(x).to(dev))
+        self.ins = [dev_t(inp[n], bf) for n in ("q", "k", "v")] + \
+                   [dev_t(inp[n], False) for n in ("i_pre", "f_pre", "C0", "n0", "m0")]
+        self.outs = [torch.empty(w.B, w.H, w.T, w.d_v, device=dev),
+                     torch.empty(w.B, w.H, w.d_v, w.d_qk, device=dev),
+                     torch.empty(w.B, w.H, w.d_qk, device=dev), torch.empty(w.B, w.H, device=dev)]
+        self.desc = capi.make_desc(w.B, w.H, w.T, w.d_qk, w.d_v,
+                                   capi.XLSTM_BF16 if bf else capi.XLSTM_F32, inp["qk_scale"], 64)
+        wsb = capi.xlstm_mlstm_workspace_size(self.desc)
+        self.ws = torch.zeros(wsb, device=dev, dtype=torch.uint8)
+        self.fn = capi.load().xlstm_mlstm_fwd_chunkwise
+        import ctypes
+        P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+        self.argv = (ctypes.byref(self.desc), *(P(t) for t in self.ins), *(P(t) for t in self.outs),
+                     P(self.ws), wsb, ctypes.c_void_p(stream.cuda_stream))
+        self.stream = stream
+        self.kernel = "chunkwise"
+        self.name = "xlstm_mlstm_fwd_chunkwise"
+
+    def step(self, i):
+        st = self.fn(*self.argv)
+        if st != 0:
+            from xlstm_mlstm_matrix_b200 import capi
+            raise capi.XlstmError(st, self.name)
+
+    def check_status(self):
+        from xlstm_mlstm_matrix_b200 import capi
+        st, where = capi.xlstm_mlstm_workspace_status(self.ws, self.stream)
+        if st != 0:
+            raise capi.XlstmError(st, f"device status (where={where})")
+
+    def host_buffers(self):
+        """Pinned host copies of the step's inputs and result buffers."""
+        import torch
+        hin = [None if t is None else t.cpu().pin_memory() for t in self.ins]
+        hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]
+        pairs_in = [(d, s) for d, s in zip(self.ins, hin) if d is not None]
+        pairs_out = list(zip(hout, self.outs))
+        return pairs_in, pairs_out
+
+
+class _Decode:
+    """One xlstm_mlstm_step per step over B*H heads, state in place in HBM."""
+
+    def __init__(self, w, inp, dev, stream):
+        import torch
+        from xlstm_mlstm_matrix_b200 import capi
+        self.w, self.inp = w, inp
+        _, C0, n0, m0 = inp["state"]
+        S = len(inp["steps"])
+        stack = lambda k: np.stack([st[k] for st in inp["steps"]])
+        bfd = lambda x: torch.from_numpy(x).to(dev).to(torch.bfloat16)
+        self.q, self.k, self.v = bfd(stack("q")), bfd(stack("k")), bfd(stack("v"))
+        self.ig = torch.from_numpy(stack("i_pre")).to(dev)
+        self.fg = torch.from_numpy(stack("f_pre")).to(dev)
+        self.C = torch.from_numpy(C0).to(dev)
+        self.n = torch.from_numpy(n0).to(dev)
+        self.m = torch.from_numpy(m0).to(dev)
+        self.h = torch.empty(w.B, w.H, w.d_v, device=dev)
+        self.S = S
+        self.desc = capi.make_desc(w.B, w.H, 1, w.d_qk, w.d_v, capi.XLSTM_BF16, inp["qk_scale"], 64)
+        self.fn = capi.load().xlstm_mlstm_step
+        import ctypes
+        self.P = lambda t: ctypes.c_void_p(t.data_ptr())
+        self.cs = ctypes.c_void_p(stream.cuda_stream)
+        self.stream = stream
+        self.kernel = "step"
+        self.name = "xlstm_mlstm_step"
+
+    def step(self, i, src=None):
+        import ctypes
+        P = self.P
+        j = i % self.S
+        q, k, v, ig, fg = src if src is not None else (self.q[j], self.k[j], self.v[j], self.ig[j],
+                                                       self.fg[j])
+        st = self.fn(ctypes.byref(self.desc), P(q), P(k), P(v), P(ig), P(fg), P(self.C), P(self.n),
+                     P(self.m), P(self.h), P(self.C), P(self.n), P(self.m), self.cs)
+        if st != 0:
+            from xlstm_mlstm_matrix_b200 import capi
+            raise capi.XlstmError(st, self.name)
+
+    def check_status(self):
+        pass
+
+    def host_buffers(self):
+        """Pinned host copies of one step's inputs (q, k, v, gates) and of h~;
+        the state stays resident on the device, as in a decode loop."""
+        import torch
+        j = 0
+        hin = [self.q[j].cpu().pin_memory(), self.k[j].cpu().pin_memory(),
+               self.v[j].cpu().pin_memory(), self.ig[j].cpu().pin_memory(),
+               self.fg[j].cpu().pin_memory()]
+        self.dev_in = [torch.empty_like(t, device=self.h.device) for t in hin]
+        pairs_in = list(zip(self.dev_in, hin))
+        pairs_out = [(torch.empty(self.h.shape, dtype=self.h.dtype).pin_memory(), self.h)]
+        return pairs_in, pairs_out
 
 
 def run_ours(args, rank, world, local_rank):
@@ -197,36 +389,10 @@ def run_ours(args, rank, world, local_rank):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     capi.load()
-    w = inputs.WORKLOADS[WORKLOAD].replace(seed=inputs.WORKLOADS[WORKLOAD].seed + 1000 * rank)
-    if args.B or args.H:   # smaller batch/head count of the same layer (profiling captures)
-        w = w.replace(B=args.B or w.B, H=args.H or w.H)
-    inp = inputs.make_sequence(w)
-    scale = inp["qk_scale"]
-    desc = capi.make_desc(w.B, w.H, w.T, w.d_qk, w.d_v, capi.XLSTM_BF16, scale, 64)
-
-    def dev_t(x, bf16):
-        t = torch.from_numpy(x).to(dev)
-        return t.to(torch.bfloat16) if bf16 else t
-
-    q, k, v = (dev_t(inp[n], True) for n in ("q", "k", "v"))
-    ig, fg = dev_t(inp["i_pre"], False), dev_t(inp["f_pre"], False)
-    h = torch.empty(w.B, w.H, w.T, w.d_v, device=dev)
-    C1 = torch.empty(w.B, w.H, w.d_v, w.d_qk, device=dev)
-    n1 = torch.empty(w.B, w.H, w.d_qk, device=dev)
-    m1 = torch.empty(w.B, w.H, device=dev)
-    wsb = capi.xlstm_mlstm_workspace_size(desc)
-    ws = torch.zeros(wsb, device=dev, dtype=torch.uint8)
+    w = workload_for_rank(args.workload, rank, args.B, args.H, args.T)
+    inp = make_inputs(w)
     stream = torch.cuda.Stream(dev)
-    fn = capi.load().xlstm_mlstm_fwd_chunkwise
-    import ctypes
-    P = lambda t: ctypes.c_void_p(t.data_ptr())
-    argv = (ctypes.byref(desc), P(q), P(k), P(v), P(ig), P(fg), None, None, None, P(h), P(C1),
-            P(n1), P(m1), P(ws), wsb, ctypes.c_void_p(stream.cuda_stream))
-
-    def step():
-        st = fn(*argv)
-        if st != 0:
-            raise capi.XlstmError(st, "xlstm_mlstm_fwd_chunkwise")
+    job = _Decode(w, inp, dev, stream) if w.steps else _Sequence(w, inp, dev, stream)
 
     dist = None
     if world > 1:
@@ -236,116 +402,115 @@ def run_ours(args, rank, world, local_rank):
         if dist is not None:
             dist.barrier()
 
-    def max_over_ranks(x):
-        if dist is None:
-            return x
-        t = torch.tensor([x], device=dev, dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+    def slowest(x):
+        return max_over_ranks(x, dist, dev)
 
     with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            step()
+        for i in range(args.warmup):
+            job.step(i)
     stream.synchronize()
-    # device status after warm-up: no bounded wait gave up
-    st, where = capi.xlstm_mlstm_workspace_status(ws, stream)
-    if st != 0:
-        raise capi.XlstmError(st, f"device status (where={where})")
+    job.check_status()          # no bounded device wait gave up during warm-up
 
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local_rank if os.environ.get("CUDA_VISIBLE_DEVICES") is None else 0) as clk:
         e0.record(stream)
-        for _ in range(args.steps):
-            step()
+        for i in range(args.steps):
+            job.step(args.warmup + i)
         e1.record(stream)
         e1.synchronize()
     torch.cuda.synchronize(dev)
     barrier()
-    ms = e0.elapsed_time(e1) / args.steps
-    ms = max_over_ranks(ms)
-    st, where = capi.xlstm_mlstm_workspace_status(ws, stream)
-    if st != 0:
-        raise capi.XlstmError(st, f"device status (where={where})")
+    ms = slowest(e0.elapsed_time(e1) / args.steps)
+    job.check_status()
 
-    tokens = w.B * w.T
-    value = world * tokens / (ms * 1e-3)
+    tokens = tokens_per_step(w)
+    value = job_rate(tokens, world, ms)
     bytes_, flops = algorithmic(w)
     hbm, bf16_peak, _, peak_src = peaks()
     achieved_gbs = bytes_ / (ms * 1e-3) / 1e9
     src_sha = kernel_source_sha()
 
     # ---- end to end: pinned host buffers through the same call ---------------------
-    hq, hk, hv = (torch.from_numpy(inp[n]).to(torch.bfloat16).pin_memory() for n in ("q", "k", "v"))
-    hig, hfg = torch.from_numpy(inp["i_pre"]).pin_memory(), torch.from_numpy(inp["f_pre"]).pin_memory()
-    oh = torch.empty(h.shape, dtype=torch.float32).pin_memory()
-    oC = torch.empty(C1.shape, dtype=torch.float32).pin_memory()
-    on = torch.empty(n1.shape, dtype=torch.float32).pin_memory()
-    om = torch.empty(m1.shape, dtype=torch.float32).pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in (hq, hk, hv, hig, hfg))
-    d2h = sum(t.numel() * t.element_size() for t in (oh, oC, on, om))
-
-    def e2e_step():
-        for dst, src in ((q, hq), (k, hk), (v, hv), (ig, hig), (fg, hfg)):
-            dst.copy_(src, non_blocking=True)
-        step()
-        for dst, src in ((oh, h), (oC, C1), (on, n1), (om, m1)):
-            dst.copy_(src, non_blocking=True)
-
-    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 5))
+    e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 5 if not w.steps else args.steps))
+    e2e = None
     if e2e_steps:
+        pairs_in, pairs_out = job.host_buffers()
+        h2d = sum(s.numel() * s.element_size() for _, s in pairs_in)
+        d2h = sum(d.numel() * d.element_size() for d, _ in pairs_out)
+
+        def e2e_step(i):
+            for dst, src in pairs_in:
+                dst.copy_(src, non_blocking=True)
+            if w.steps:
+                job.step(i, src=[d for d, _ in pairs_in])
+            else:
+                job.step(i)
+            for dst, src in pairs_out:
+                dst.copy_(src, non_blocking=True)
+
         with torch.cuda.stream(stream):
-            e2e_step()
+            e2e_step(0)
             stream.synchronize()
             barrier()
             e0.record(stream)
-            for _ in range(e2e_steps):
-                e2e_step()
+            for i in range(e2e_steps):
+                e2e_step(i)
             e1.record(stream)
             e1.synchronize()
         barrier()
-    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / e2e_steps) if e2e_steps else None
+        e2e_ms = slowest(e0.elapsed_time(e1) / e2e_steps)
+        e2e = {"value": job_rate(tokens, world, e2e_ms), "unit": UNIT,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+        if w.steps:
+            e2e["note"] = "per step: H2D of q, k, v and gates, D2H of h~; state resident on the device"
+        job.check_status()
 
     if rank == 0:
+        l2 = (f"inputs larger than L2 ({bytes_ / 1e9:.2f} GB per step vs 126 MB L2)"
+              if bytes_ > 4 * 126e6 else "working set near L2 size; no flush")
+        extra = {"inputs": "bf16 q/k/v, fp32 gates; fp32 h and state", "l2": l2,
+                 "parallelism": f"replicas x{world} (independent heads)"}
+        if not w.steps:
+            extra["chunk"] = 64
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-            "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "T": w.T, "d_qk": w.d_qk,
-                       "d_v": w.d_v, "chunk": 64, "inputs": "bf16 q/k/v, fp32 gates; fp32 h and state",
-                       "l2": "inputs larger than L2 (1.1 GB per step vs 126 MB L2)",
-                       "parallelism": f"replicas x{world} (independent heads)"},
+            "config": config_of(w, extra),
             "tflops": world * flops / (ms * 1e-3) / 1e12,
             "hbm_gbs": achieved_gbs,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved_gbs / hbm, "traffic": traffic_for(src_sha),
-                         "peak_source": peak_src,
+                         "frac": achieved_gbs / hbm, "traffic": traffic_for(src_sha, w.name),
+                         "peak_source": peak_src, "kernel": job.kernel,
                          "algorithmic_bytes_per_launch": bytes_, "flops_per_launch": flops,
                          "tensor_frac": flops / (ms * 1e-3) / 1e12 / bf16_peak},
             "gpu_launches": args.steps,
-            "e2e": None if e2e_ms is None else {
-                "value": world * tokens / (e2e_ms * 1e-3), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "e2e": e2e,
             "clocks": clk.summary(),
             "kernel_source_sha": src_sha,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(inp, budget_s=args.ref_budget)
+            line["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.ref_budget)
         print(json.dumps(line), flush=True)
 
 
 def main():
+    from xlstm_mlstm_matrix_b200.inputs import WORKLOADS
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=[k for k in WORKLOADS if k != "tiny_fp32"],
+                    default=DEFAULT_WORKLOAD)
     ap.add_argument("--ref-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
     ap.add_argument("--H", type=int, default=0, help="override the head count (profiling)")
+    ap.add_argument("--T", type=int, default=0, help="override the sequence length (profiling)")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
     rank = int(os.environ.get("RANK", 0))

@@ -27,8 +27,17 @@ def gpu_sequence(inp: dict, kind: str, chunk: int = 0, qk_scale=None, state=None
     if state is None and inp.get("C0") is not None:
         state = tuple(to_dev(inp[n], "f32") for n in ("C0", "n0", "m0"))
     scale = inp["qk_scale"] if qk_scale is None else qk_scale
-    h, (C, n, m) = capi.fwd(q, k, v, ig, fg, state=state, qk_scale=scale, chunk=chunk, kind=kind)
+    ws = None
+    if kind == "chunkwise":
+        B, H, T, dqk = q.shape
+        desc = capi.make_desc(B, H, T, dqk, v.shape[-1], capi.XLSTM_BF16 if dt == "bf16" else capi.XLSTM_F32,
+                              scale, chunk)
+        ws = torch.zeros(max(256, capi.xlstm_mlstm_workspace_size(desc)), device=q.device, dtype=torch.uint8)
+    h, (C, n, m) = capi.fwd(q, k, v, ig, fg, state=state, qk_scale=scale, chunk=chunk, kind=kind, workspace=ws)
     torch.cuda.synchronize()
+    if ws is not None:   # no bounded device wait gave up
+        code, where = capi.xlstm_mlstm_workspace_status(ws)
+        assert code == capi.XLSTM_OK, f"device status {capi.xlstm_status_string(code)} (wait {where})"
     return h.cpu().numpy(), C.cpu().numpy(), n.cpu().numpy(), m.cpu().numpy()
 
 
