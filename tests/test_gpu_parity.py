@@ -100,6 +100,21 @@ def test_stabilizer_stress(gate, mean_i, std_i, dtype, dv):
         compare(gpu_sequence(inp, kind), ref, dtype, f"{kind} {gate}", row_tol=tol)
 
 
+@pytest.mark.parametrize("dqk,dv", [(64, 128), (256, 128)])
+def test_exact_and_fast_chunks_alternating_repeated(dqk, dv):
+    """Input-gate jumps far beyond the fast path's range make exact and fast chunks
+    alternate; the hand-offs between the two kinds of chunk must hold however the
+    warps are timed, so the same call runs many times and every run must finish
+    with a clean device status and the same result."""
+    inp = small_inputs(2, 2, 300, dqk, dv, "bf16", True, seed=11, gate="std", mean_i=30.0, std_i=40.0)
+    ref = oracle_sequence(inp)
+    first = gpu_sequence(inp, "chunkwise")
+    compare(first, ref, "bf16", "alternating exact/fast", row_tol=fp32_row_tolerance(inp))
+    for _ in range(24):
+        got = gpu_sequence(inp, "chunkwise")   # asserts a clean device status
+        np.testing.assert_array_equal(got[0], first[0])
+
+
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
 @pytest.mark.parametrize("dv", [64, 128])
 def test_reset_gates(dtype, dv):

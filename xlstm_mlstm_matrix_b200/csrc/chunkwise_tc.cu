@@ -38,7 +38,8 @@
 // memory is full (C_acc 256 + C_hi 128 + H 64 + S 64 columns) and C_lo goes
 // through a 32 KB shared half-buffer, refilled while the first half is read.
 //
-// Warps: 0 TMA producer, 1 MMA issuer (owns TMEM), 2 gate scan, 3 normaliser,
+// Warps: 0 TMA producer (and L2 prefetch two chunks ahead), 1 MMA issuer (owns
+// TMEM), 2 gate scan, 3 normaliser,
 // 4-7 state group (lower half of the state split, epilogue), 8-11 token group
 // (w V, upper half of the state split, n.q, P).
 // Every wait is bounded: one that gives up records XLSTM_ERR_TIMEOUT in the
@@ -95,8 +96,11 @@ struct Cfg {
     // gate ring: per slot UH, UL, MH, ML, AH, AN, W, LOWER [64] + 8 chunk scalars
     static constexpr int G_FLOATS = 8 * kL + 8;
     static constexpr int OFF_G = OFF_CLO + CLO_BYTES;
-    static constexpr int OFF_N = OFF_G + kNG * G_FLOATS * 4;   // n_acc double buffer
-    static constexpr int OFF_SC = OFF_N + 2 * DQK * 4;          // nq, rsum, inv, coef [2][64] each
+    // n_acc double buffer; the upper half of the columns sits 16 bytes further on so
+    // that the two threads of a token (one per half) read from different banks
+    static constexpr int NBUF = DQK + 4;
+    static constexpr int OFF_N = OFF_G + kNG * G_FLOATS * 4;
+    static constexpr int OFF_SC = OFF_N + 2 * NBUF * 4;         // nq, rsum, inv, coef [2][64] each
     static constexpr int OFF_BAR = OFF_SC + 8 * kL * 4;
     static constexpr int NBARS = 32;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
@@ -121,7 +125,10 @@ enum : int { kSRho = 0, kSRescale = 1, kSExact = 2, kSMEnd = 3, kSGsc = 4 };
 // Barriers.
 enum : int {
     B_KV_FULL = 0, B_KV_EMPTY = 2, B_Q_FULL = 4, B_Q_EMPTY = 6, B_G_FULL = 8, B_G_EMPTY = B_G_FULL + kNG,
-    B_S_FULL = B_G_EMPTY + kNG, B_S_EMPTY, B_OPS, B_VT, B_CONV0, B_CONV1, B_CLO_FREE, B_H_FULL, B_H_EMPTY,
+    // B_VT: w V is in place for a fast chunk (token group); B_VT_EXACT: the gauge
+    // move and w V of an exact chunk are done (state group).  Two producers on one
+    // barrier could complete two phases before the MMA warp waits for the first.
+    B_S_FULL = B_G_EMPTY + kNG, B_S_EMPTY, B_OPS, B_VT, B_VT_EXACT, B_CONV0, B_CONV1, B_CLO_FREE, B_H_FULL, B_H_EMPTY,
     B_UPD_DONE, B_N_READY, B_N_FREE = B_N_READY + 2, B_DRAIN = B_N_FREE + 2, B_COUNT
 };
 static_assert(B_COUNT <= 32, "barrier space");
@@ -199,6 +206,10 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, u
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u) {
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
+
+// Padded index of column j in an n buffer.
+template <int DQK>
+__device__ __forceinline__ int nidx(int j) { return j + (j >= DQK / 2 ? 4 : 0); }
 
 // x -> (hi, lo) float pair with hi + lo = x to ~2^-48; -inf -> (-inf, 0).
 __device__ __forceinline__ void split_double(double x, float &hi, float &lo) {
@@ -304,7 +315,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar[B_N_READY + i], 1); mbar_init(&bar[B_N_FREE + i], 1);
         }
         for (int i = 0; i < kNG; ++i) { mbar_init(&bar[B_G_FULL + i], 1); mbar_init(&bar[B_G_EMPTY + i], 3); }
-        const int ones[] = {B_S_FULL, B_S_EMPTY, B_OPS, B_VT, B_CONV1, B_CLO_FREE, B_H_FULL, B_H_EMPTY,
+        const int ones[] = {B_S_FULL, B_S_EMPTY, B_OPS, B_VT, B_VT_EXACT, B_CONV1, B_CLO_FREE, B_H_FULL, B_H_EMPTY,
                             B_UPD_DONE, B_DRAIN};
         mbar_init(&bar[B_CONV0], 2);   // both compute groups split half of the state
         for (int b : ones) mbar_init(&bar[b], 1);
@@ -328,6 +339,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             int kv_issued[2] = {0, 0}, q_issued[2] = {0, 0};
             for (int c = 0; c < NC; ++c) {
                 const int s = c & 1;
+                if (c + 2 < NC) {   // chunk c+2 into L2 now, so that its stage load hits L2 later
+                    for (int b = 0; b < C::NKB; ++b) {
+                        tma_prefetch_l2_3d(&tmk, 64 * b, kL * (c + 2), bh);
+                        tma_prefetch_l2_3d(&tmq, 64 * b, kL * (c + 2), bh);
+                    }
+                    for (int b = 0; b < 2; ++b) tma_prefetch_l2_3d(&tmv, v0 + 64 * b, kL * (c + 2), bh);
+                }
                 if (c >= 2 && !wait1(sh, &bar[B_KV_EMPTY + s], ((c >> 1) - 1) & 1, kWhereTmaKvEmpty)) break;
                 mbar_arrive_expect_tx(&bar[B_KV_FULL + s], C::K_BYTES + C::V_BYTES);
                 uint8_t *Ks = sm + C::OFF_K + s * C::K_BYTES;
@@ -356,6 +374,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t idU = make_idesc(128, DQK, kFmtBF16, kFmtBF16, 1, 1);
             const uint32_t p_addr = smem_u32(Ps), clo_addr = smem_u32(sm + C::OFF_CLO);
             bool issued = false, prev_exact = false;
+            int nfast = 0, nexact = 0;   // phases of B_VT and B_VT_EXACT consumed
             for (int c = 0; c < NC; ++c) {
                 const int s = c & 1, slot = c % kNG;
                 const uint32_t q_addr = smem_u32(sm + C::OFF_Q + s * C::Q_BYTES);
@@ -379,33 +398,40 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const bool exact = gring[slot * C::G_FLOATS + kGScal + kSExact] != 0.f;
                 if (!wait1(sh, &bar[B_CONV0], c & 1, kWhereMmaConv)) break;
                 if (!wait1(sh, &bar[B_OPS], c & 1, kWhereMmaOps)) break;
-                if (!exact && !wait1(sh, &bar[B_VT], c & 1, kWhereMmaVt)) break;
+                if (!exact && !wait1(sh, &bar[B_VT], (nfast++) & 1, kWhereMmaVt)) break;
                 if (c >= 1 && !prev_exact && !wait1(sh, &bar[B_H_EMPTY], (c - 1) & 1, kWhereMmaHEmpty)) break;
                 tc_fence_after();
                 // H = C_hi Q^T + C_lo Q^T
-#pragma unroll
-                for (int ks = 0; ks < DQK / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_f16_ts(tm + C::TM_H, tm + C::TM_CHI + 8 * ks, smem_desc_sw128(q_addr + off, 16, 1024),
-                               idR, ks > 0);
-                }
                 if (C::BIG) {
-                    for (int hf = 0; hf < 2; ++hf) {
-                        if (hf == 1) {
-                            tc_commit(&bar[B_CLO_FREE]);
-                            if (!wait1(sh, &bar[B_CONV1], c & 1, kWhereMmaClo)) goto mma_done;
-                            tc_fence_after();
-                        }
+                    // C_lo of the lower half first (its shared tile is complete at conv0), then
+                    // release the tile, so that the token group refills it with the upper half
+                    // while the C_hi MMAs run
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const int ks = 8 * hf + kk;
-                            const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-                            mma_f16_ss(tm + C::TM_H,
-                                       smem_desc_sw128(clo_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                       smem_desc_sw128(q_addr + off, 16, 1024), idR, 1);
-                        }
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_f16_ss(tm + C::TM_H, smem_desc_sw128(clo_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                   smem_desc_sw128(q_addr + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), idR, kk > 0);
+                    tc_commit(&bar[B_CLO_FREE]);
+#pragma unroll
+                    for (int ks = 0; ks < DQK / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        mma_f16_ts(tm + C::TM_H, tm + C::TM_CHI + 8 * ks, smem_desc_sw128(q_addr + off, 16, 1024),
+                                   idR, 1);
+                    }
+                    if (!wait1(sh, &bar[B_CONV1], c & 1, kWhereMmaClo)) break;
+                    tc_fence_after();
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const int ks = 8 + kk;
+                        mma_f16_ss(tm + C::TM_H, smem_desc_sw128(clo_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                                   smem_desc_sw128(q_addr + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), idR, 1);
                     }
                 } else {
+#pragma unroll
+                    for (int ks = 0; ks < DQK / 16; ++ks) {
+                        const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
+                        mma_f16_ts(tm + C::TM_H, tm + C::TM_CHI + 8 * ks, smem_desc_sw128(q_addr + off, 16, 1024),
+                                   idR, ks > 0);
+                    }
 #pragma unroll
                     for (int ks = 0; ks < DQK / 16; ++ks) {
                         const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
@@ -426,7 +452,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_commit(&bar[B_H_FULL]);
                 tc_commit(&bar[B_Q_EMPTY + s]);
                 if (exact) {
-                    if (!wait1(sh, &bar[B_VT], c & 1, kWhereMmaVt)) break;
+                    if (!wait1(sh, &bar[B_VT_EXACT], (nexact++) & 1, kWhereMmaVt)) break;
                     tc_fence_after();
                 }
                 // C_acc += (w V)^T K
@@ -438,7 +464,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_commit(&bar[B_KV_EMPTY + s]);
                 prev_exact = exact;
             }
-        mma_done:
             if (issued) {   // drain: all issued MMAs complete before tensor memory is freed
                 tc_commit(&bar[B_DRAIN]);
                 drain_wait(&bar[B_DRAIN], 0);
@@ -518,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int i = 0; i < NPL; ++i) nacc[i] = p.n0 ? p.n0[(size_t)bh * DQK + j0 + i] : 0.f;
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) nbuf[j0 + i] = nacc[i];
+        for (int i = 0; i < NPL; ++i) nbuf[nidx<DQK>(j0 + i)] = nacc[i];
         __syncwarp();
         if (lane == 0) mbar_arrive(&bar[B_N_READY]);
         float gsc = 1.f;
@@ -559,7 +584,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nb = (c + 1) & 1;
             if (c >= 1 && !waitw(sh, &bar[B_N_FREE + nb], ((c - 1) >> 1) & 1, kWhereNormFree)) { alive = false; break; }
 #pragma unroll
-            for (int i = 0; i < NPL; ++i) nbuf[nb * DQK + j0 + i] = nacc[i];
+            for (int i = 0; i < NPL; ++i) nbuf[nb * C::NBUF + nidx<DQK>(j0 + i)] = nacc[i];
             __syncwarp();
             if (lane == 0) {
                 mbar_arrive(&bar[B_N_READY + nb]);
@@ -642,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
             named_barrier(1, 128);   // unconditional: every warp of the group takes every barrier
-            if (st == 0 && alive && exact) mbar_arrive(&bar[B_VT]);
+            if (st == 0 && alive && exact) mbar_arrive(&bar[B_VT_EXACT]);
             // --- epilogue: h~[t][v] = (AH_t H[v][t] (+ intra[v][t])) / den_t
             if (alive) {
                 const int len = min(kL, T - kL * c);
@@ -747,7 +772,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             alive = alive && waitw(sh, &bar[B_N_READY + (c & 1)], (c >> 1) & 1, kWhereTkN);
             if (alive) {
                 const uint8_t *Qs = sm + C::OFF_Q + s * C::Q_BYTES;
-                const float *nn = nbuf + (c & 1) * DQK;
+                const float *nn = nbuf + (c & 1) * C::NBUF + (half ? 4 : 0);
                 float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
                                  make_float2(0.f, 0.f)};
 #pragma unroll 1
@@ -756,7 +781,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     float4 na[4], nb[4];
 #pragma unroll
                     for (int k4 = 0; k4 < 4; ++k4) {
-                        const int j = half * (DQK / 2) + 8 * (g0 + k4);
+                        // the upper-half thread walks its chunks rotated by 4 so that the
+                        // pair of a token hits distinct banks
+                        const int ci = half ? (g0 + k4 + 4) % (DQK / 16) : g0 + k4;
+                        const int j = half * (DQK / 2) + 8 * ci;
                         u[k4] = *reinterpret_cast<const uint4 *>(Qs + (j >> 6) * 8192 + sw128_offset(trow, (j & 63) >> 3));
                         na[k4] = *reinterpret_cast<const float4 *>(nn + j);
                         nb[k4] = *reinterpret_cast<const float4 *>(nn + j + 4);
@@ -782,15 +810,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             alive = alive && waitw(sh, &bar[B_S_FULL], c & 1, kWhereTkS);
             if (alive) {
                 tc_fence_after();
-                float r0[32], r1[32];
-                tmem_ld32(tm + lane_base + C::TM_S, r0);
-                tmem_ld32(tm + lane_base + C::TM_S + 32, r1);
+                float r0[32];   // lanes l and l + 16: columns [0, 32) and [32, 64) of row 16 wq + (l & 15)
+                tmem_ld16x2_32(tm + lane_base + C::TM_S, r0);
                 tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 32; ++i) {
-                    const float up = __shfl_sync(0xffffffffu, r1[i], lane & 15);
-                    if (lane >= 16) r0[i] = up;
-                }
                 const int t = 16 * wq + (lane & 15);
                 const int s0 = 32 * (lane >> 4);
                 float rs = 0.f;
