@@ -69,7 +69,7 @@ enum : int32_t {
     kWhereTmaKvEmpty = 1, kWhereTmaQEmpty, kWhereMmaKvFull, kWhereMmaQFull, kWhereMmaSEmpty, kWhereMmaGate,
     kWhereMmaConv, kWhereMmaOps, kWhereMmaVt, kWhereMmaHEmpty, kWhereMmaClo, kWhereGateEmpty, kWhereNormGate,
     kWhereNormKv, kWhereNormFree, kWhereStUpd, kWhereStGate, kWhereStClo, kWhereStOps, kWhereStH, kWhereStFinal,
-    kWhereTkH, kWhereTkGate, kWhereTkKv, kWhereTkQ, kWhereTkN, kWhereTkS, kWhereTkUpd, kWhereTkClo
+    kWhereTkH, kWhereTkGate, kWhereTkKv, kWhereTkQ, kWhereTkN, kWhereTkS, kWhereTkUpd, kWhereTkClo, kWhereTkConv
 };
 
 // Test hook: make the gate warp withhold one hand-off so that its consumers time out.
@@ -154,8 +154,8 @@ __device__ __forceinline__ void record_timeout(const Shared &sh, int where) {
 }
 
 // Single-thread bounded wait; gives up on timeout or when another role aborted.
-__device__ __forceinline__ bool wait1(const Shared &sh, uint64_t *bar, uint32_t parity, int where) {
-    if (mbar_try_wait(bar, parity)) return true;
+// Only the first test is inlined at the call sites; the waiting loop exists once.
+__device__ __noinline__ bool wait1_slow(const Shared &sh, uint64_t *bar, uint32_t parity, int where) {
     const uint64_t t0 = global_timer_ns();
     for (;;) {
         // suspended in hardware (no issue slots) until the phase completes or 20 us pass
@@ -166,6 +166,9 @@ __device__ __forceinline__ bool wait1(const Shared &sh, uint64_t *bar, uint32_t 
             return false;
         }
     }
+}
+__device__ __forceinline__ bool wait1(const Shared &sh, uint64_t *bar, uint32_t parity, int where) {
+    return mbar_try_wait(bar, parity) || wait1_slow(sh, bar, parity, where);
 }
 // Whole-warp bounded wait: every lane agrees on the outcome.
 __device__ __forceinline__ bool waitw(const Shared &sh, uint64_t *bar, uint32_t parity, int where) {
@@ -206,6 +209,11 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, u
 __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u) {
     return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
 }
+
+// Descriptor offsets (16-byte units) of K-step ks in a K-major 128B-swizzled tile of
+// 64-column boxes: boxes 8 KB apart for q / k tiles, 16 KB apart for the C_lo tile.
+__device__ __forceinline__ uint32_t kstep(int ks) { return (uint32_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4); }
+__device__ __forceinline__ uint32_t cstep(int ks) { return (uint32_t)(((ks >> 2) * 16384 + (ks & 3) * 32) >> 4); }
 
 // Padded index of column j in an n buffer.
 template <int DQK>
@@ -255,11 +263,8 @@ __device__ __forceinline__ void load32(const float *src, float (&d)[32]) {
 // lo_mode: 0 C_hi and C_lo to TMEM; 1 C_hi to TMEM, C_lo to the shared tile at
 // local column jlo; 2 C_hi only; 3 C_lo only (shared tile, no gauge move).
 template <class C>
-__device__ __forceinline__ void split_state_block(uint32_t tm, uint32_t lane_base, int i, bool mv, float rho,
-                                                  int lo_mode, uint8_t *clo_s, int row, int jlo) {
-    float r[32];
-    tmem_ld32(tm + lane_base + C::TM_C + 32 * i, r);
-    tmem_wait_ld();
+__device__ __forceinline__ void split_state_block(float (&r)[32], uint32_t tm, uint32_t lane_base, int i, bool mv,
+                                                  float rho, int lo_mode, uint8_t *clo_s, int row, int jlo) {
     if (mv) {
 #pragma unroll
         for (int x = 0; x < 32; x += 2) {
@@ -280,6 +285,135 @@ __device__ __forceinline__ void split_state_block(uint32_t tm, uint32_t lane_bas
             const int j = jlo + 8 * q4;
             *reinterpret_cast<uint4 *>(clo_s + (j >> 6) * 16384 + sw128_offset(row, (j & 63) >> 3)) =
                 make_uint4(lo[4 * q4], lo[4 * q4 + 1], lo[4 * q4 + 2], lo[4 * q4 + 3]);
+        }
+    }
+}
+
+// ---- exact-chunk paths (rare: the stabilizer jumps inside the chunk), kept out of
+// line so that the per-chunk code of the fast path stays compact in the
+// instruction cache.
+
+// C_acc *= rho over this thread's row (gauge move to r = mu_L), then V <- w V.
+template <class C>
+__device__ __noinline__ void exact_gauge_move_and_scale_v(uint32_t tm, uint32_t lane_base, float rho, uint8_t *Vs,
+                                                          const float *w, int t128) {
+    float r[32];
+#pragma unroll 1
+    for (int i = 0; i < C::NKB * 2; ++i) {
+        tmem_ld32(tm + lane_base + C::TM_C + 32 * i, r);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) r[x] *= rho;
+        tmem_st32(tm + lane_base + C::TM_C + 32 * i, r);
+    }
+    tmem_wait_st();
+    scale_v_rows(Vs, w, t128);
+}
+
+// Epilogue of an exact chunk: h~ = coef_t H + inv_t intra, both 32-token halves.
+template <class C>
+__device__ __noinline__ void exact_epilogue(uint32_t tm, uint32_t lane_base, const float *coef, const float *inv,
+                                            float *hc, size_t dv, int len) {
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {
+        float rh[32], ra[32], cf[32];
+        tmem_ld32(tm + lane_base + C::TM_H + 32 * hh, rh);
+        tmem_ld32(tm + lane_base + C::TM_S + 32 * hh, ra);
+        load32(coef + 32 * hh, cf);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) rh[x] *= cf[x];
+        load32(inv + 32 * hh, cf);
+#pragma unroll
+        for (int x = 0; x < 32; ++x) rh[x] = fmaf(ra[x], cf[x], rh[x]);
+        float *hrow = hc + (size_t)32 * hh * dv;
+        const int n = min(32, len - 32 * hh);
+#pragma unroll 1
+        for (int x = 0; x < n; ++x) hrow[(size_t)x * dv] = rh[x];
+    }
+}
+
+// 2^e for e <= 0 with the hardware's approximate exponential (relative error far
+// below the 2^-16 of the bf16 hi/lo operands it feeds; 2^e below 2^-126 flushes to 0).
+__device__ __forceinline__ float ex2_approx(float e) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(e));
+    return y;
+}
+
+// P rows of one thread (hi / lo, K-major 128B-swizzled) and the row sum.
+__device__ __forceinline__ void store_p_row(const float (&r0)[32], uint8_t *Ps, float *rs, float rsum, int t,
+                                            int lane) {
+#pragma unroll
+    for (int ch = 0; ch < 4; ++ch) {
+        uint32_t hi[4], lo[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) split_bf16x2(r0[8 * ch + 2 * i], r0[8 * ch + 2 * i + 1], hi[i], lo[i]);
+        const int chunk = 4 * (lane >> 4) + ch;
+        *reinterpret_cast<uint4 *>(Ps + sw128_offset(t, chunk)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        *reinterpret_cast<uint4 *>(Ps + 8192 + sw128_offset(t, chunk)) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+    }
+    rsum += __shfl_xor_sync(0xffffffffu, rsum, 16);
+    if (lane < 16) rs[t] = rsum;
+}
+
+// P of a fast chunk from S (M = 64: token row 16 wq + (l & 15) in lane l & 15 of each
+// quarter; lanes l and l + 16 take columns [0, 32) and [32, 64) of that row): the
+// causal mask, and the row sum of mask(S) w times AH_t.
+__device__ __forceinline__ void p_pass(uint32_t s_tmem, const float *g, uint8_t *Ps, float *rs, int wq, int lane) {
+    float r0[32];
+    tmem_ld16x2_32(s_tmem, r0);
+    tmem_wait_ld();
+    const int t = 16 * wq + (lane & 15);
+    const int s0 = 32 * (lane >> 4);
+    float ww[32];
+    load32(g + kGW + s0, ww);
+    float2 r2 = make_float2(0.f, 0.f);
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        r0[i] = (s0 + i <= t) ? r0[i] : 0.f;
+        r0[i + 1] = (s0 + i + 1 <= t) ? r0[i + 1] : 0.f;
+        r2 = __ffma2_rn(make_float2(r0[i], r0[i + 1]), make_float2(ww[i], ww[i + 1]), r2);
+    }
+    store_p_row(r0, Ps, rs, g[kGAH + t] * (r2.x + r2.y), t, lane);
+}
+
+// Exact chunk: P_ts = scale S_ts e^{u_s - mu_t} for s <= t (every exponent <= 0,
+// from the float hi/lo pairs) and the plain row sums.
+__device__ __noinline__ void exact_p_pass(uint32_t s_tmem, const float *g, uint8_t *Ps, float *rs, float scale,
+                                          int wq, int lane) {
+    float r0[32];
+    tmem_ld16x2_32(s_tmem, r0);
+    tmem_wait_ld();
+    const int t = 16 * wq + (lane & 15);
+    const int s0 = 32 * (lane >> 4);
+    const float mh = g[kGMh + t], ml = g[kGMl + t];
+    float rsum = 0.f;
+#pragma unroll
+    for (int i = 0; i < 32; ++i) {
+        const float e = (g[kGUh + s0 + i] - mh) + (g[kGUl + s0 + i] - ml);
+        r0[i] = (s0 + i <= t) ? scale * r0[i] * ex2_approx(e) : 0.f;
+        rsum += r0[i];
+    }
+    store_p_row(r0, Ps, rs, rsum, t, lane);
+}
+
+// Blocks [i0, i1) of this thread's C_acc row through split_state_block, with the
+// next block's tensor-memory load in flight while a block is split.
+template <class C>
+__device__ __forceinline__ void split_range(uint32_t tm, uint32_t lane_base, int i0, int i1, bool mv, float rho,
+                                            int lo_mode, uint8_t *clo_s, int row, int jlo0) {
+    float ra[32], rb[32];
+    tmem_ld32(tm + lane_base + C::TM_C + 32 * i0, ra);
+#pragma unroll 1
+    for (int i = i0; i < i1; i += 2) {
+        tmem_wait_ld();
+        if (i + 1 < i1) tmem_ld32(tm + lane_base + C::TM_C + 32 * (i + 1), rb);
+        split_state_block<C>(ra, tm, lane_base, i, mv, rho, lo_mode, clo_s, row, jlo0 + 32 * (i - i0));
+        if (i + 1 < i1) {
+            tmem_wait_ld();
+            if (i + 2 < i1) tmem_ld32(tm + lane_base + C::TM_C + 32 * (i + 2), ra);
+            split_state_block<C>(rb, tm, lane_base, i + 1, mv, rho, lo_mode, clo_s, row, jlo0 + 32 * (i + 1 - i0));
         }
     }
 }
@@ -385,13 +519,17 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (c >= 1 && !wait1(sh, &bar[B_S_EMPTY], (c - 1) & 1, kWhereMmaSEmpty)) break;
                 if (c >= 1 && prev_exact && !wait1(sh, &bar[B_H_EMPTY], (c - 1) & 1, kWhereMmaHEmpty)) break;
                 tc_fence_after();
+                // Descriptors are built once per chunk and advanced by K-step offsets (in
+                // 16-byte units; shared addresses stay below 2^18, so the address field of
+                // a descriptor never carries).  The issue loops stay rolled: the MMA warp is
+                // not instruction-bound, and compact code keeps the instruction cache free
+                // for the compute warps.
+                const uint64_t dq = smem_desc_sw128(q_addr, 16, 1024), dk = smem_desc_sw128(k_addr, 16, 1024);
+                const uint64_t dv_mn = smem_desc_sw128(v_addr, 8192, 1024), dk_mn = smem_desc_sw128(k_addr, 8192, 1024);
                 // S = Q K^T
-#pragma unroll
-                for (int ks = 0; ks < DQK / 16; ++ks) {
-                    const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-                    mma_f16_ss(tm + C::TM_S, smem_desc_sw128(q_addr + off, 16, 1024),
-                               smem_desc_sw128(k_addr + off, 16, 1024), idS, ks > 0);
-                }
+#pragma unroll 1
+                for (int ks = 0; ks < DQK / 16; ++ks)
+                    mma_f16_ss(tm + C::TM_S, dq + kstep(ks), dk + kstep(ks), idS, ks > 0);
                 issued = true;
                 tc_commit(&bar[B_S_FULL]);
                 if (!wait1(sh, &bar[B_G_FULL + slot], (c / kNG) & 1, kWhereMmaGate)) break;
@@ -406,49 +544,39 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // C_lo of the lower half first (its shared tile is complete at conv0), then
                     // release the tile, so that the token group refills it with the upper half
                     // while the C_hi MMAs run
-#pragma unroll
+                    const uint64_t dclo = smem_desc_sw128(clo_addr, 16, 1024);   // [2 boxes][128 rows][128 B]
+#pragma unroll 1
                     for (int kk = 0; kk < 8; ++kk)
-                        mma_f16_ss(tm + C::TM_H, smem_desc_sw128(clo_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                   smem_desc_sw128(q_addr + (kk >> 2) * 8192 + (kk & 3) * 32, 16, 1024), idR, kk > 0);
+                        mma_f16_ss(tm + C::TM_H, dclo + cstep(kk), dq + kstep(kk), idR, kk > 0);
                     tc_commit(&bar[B_CLO_FREE]);
-#pragma unroll
-                    for (int ks = 0; ks < DQK / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-                        mma_f16_ts(tm + C::TM_H, tm + C::TM_CHI + 8 * ks, smem_desc_sw128(q_addr + off, 16, 1024),
-                                   idR, 1);
-                    }
+#pragma unroll 1
+                    for (int ks = 0; ks < DQK / 16; ++ks)
+                        mma_f16_ts(tm + C::TM_H, tm + C::TM_CHI + 8 * ks, dq + kstep(ks), idR, 1);
                     if (!wait1(sh, &bar[B_CONV1], c & 1, kWhereMmaClo)) break;
                     tc_fence_after();
-#pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const int ks = 8 + kk;
-                        mma_f16_ss(tm + C::TM_H, smem_desc_sw128(clo_addr + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                                   smem_desc_sw128(q_addr + (ks >> 2) * 8192 + (ks & 3) * 32, 16, 1024), idR, 1);
-                    }
+#pragma unroll 1
+                    for (int kk = 0; kk < 8; ++kk)
+                        mma_f16_ss(tm + C::TM_H, dclo + cstep(kk), dq + kstep(8 + kk), idR, 1);
                 } else {
-#pragma unroll
-                    for (int ks = 0; ks < DQK / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-                        mma_f16_ts(tm + C::TM_H, tm + C::TM_CHI + 8 * ks, smem_desc_sw128(q_addr + off, 16, 1024),
-                                   idR, ks > 0);
-                    }
-#pragma unroll
-                    for (int ks = 0; ks < DQK / 16; ++ks) {
-                        const uint32_t off = (ks >> 2) * 8192 + (ks & 3) * 32;
-                        mma_f16_ts(tm + C::TM_H, tm + C::TM_CLO + 8 * ks, smem_desc_sw128(q_addr + off, 16, 1024),
-                                   idR, 1);
-                    }
+#pragma unroll 1
+                    for (int ks = 0; ks < DQK / 16; ++ks)
+                        mma_f16_ts(tm + C::TM_H, tm + C::TM_CHI + 8 * ks, dq + kstep(ks), idR, ks > 0);
+#pragma unroll 1
+                    for (int ks = 0; ks < DQK / 16; ++ks)
+                        mma_f16_ts(tm + C::TM_H, tm + C::TM_CLO + 8 * ks, dq + kstep(ks), idR, 1);
                 }
                 // intra part: fast chunks accumulate (w V)^T (mask S)^T onto H; exact
                 // chunks put V^T P^T into the S columns
-#pragma unroll
-                for (int part = 0; part < 2; ++part)
-#pragma unroll
-                    for (int ks = 0; ks < kL / 16; ++ks)
-                        mma_f16_ss(exact ? tm + C::TM_S : tm + C::TM_H,
-                                   smem_desc_sw128(v_addr + ks * 2048, 8192, 1024),
-                                   smem_desc_sw128(p_addr + part * 8192 + ks * 32, 16, 1024), idPV,
-                                   exact ? (uint32_t)((part | ks) != 0) : 1u);
+                {
+                    const uint64_t dp = smem_desc_sw128(p_addr, 16, 1024);
+                    const uint32_t dst = exact ? tm + C::TM_S : tm + C::TM_H;
+#pragma unroll 1
+                    for (int i = 0; i < 2 * (kL / 16); ++i) {   // P_hi then P_lo, K = 16 tokens each
+                        const int part = i >> 2, ks = i & 3;
+                        mma_f16_ss(dst, dv_mn + (uint32_t)(ks * 2048 >> 4), dp + (uint32_t)((part * 8192 + ks * 32) >> 4),
+                                   idPV, exact ? (uint32_t)(i != 0) : 1u);
+                    }
+                }
                 tc_commit(&bar[B_H_FULL]);
                 tc_commit(&bar[B_Q_EMPTY + s]);
                 if (exact) {
@@ -456,10 +584,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                     tc_fence_after();
                 }
                 // C_acc += (w V)^T K
-#pragma unroll
+#pragma unroll 1
                 for (int ks = 0; ks < kL / 16; ++ks)
-                    mma_f16_ss(tm + C::TM_C, smem_desc_sw128(v_addr + ks * 2048, 8192, 1024),
-                               smem_desc_sw128(k_addr + ks * 2048, 8192, 1024), idU, 1);
+                    mma_f16_ss(tm + C::TM_C, dv_mn + (uint32_t)(ks * 2048 >> 4), dk_mn + (uint32_t)(ks * 2048 >> 4),
+                               idU, 1);
                 tc_commit(&bar[B_UPD_DONE]);
                 tc_commit(&bar[B_KV_EMPTY + s]);
                 prev_exact = exact;
@@ -629,9 +757,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const bool mv = !exact && g[kGScal + kSRescale] != 0.f;
                 const float rho = g[kGScal + kSRho];
-#pragma unroll 1
-                for (int i = 0; i < DQK / 64; ++i)
-                    split_state_block<C>(tm, lane_base, i, mv, rho, C::BIG ? 1 : 0, clo_s, st, 32 * i);
+                split_range<C>(tm, lane_base, 0, DQK / 64, mv, rho, C::BIG ? 1 : 0, clo_s, st, 0);
                 tmem_wait_st();
                 if (C::BIG) fence_proxy_async_smem();
                 tc_fence_before();
@@ -650,18 +776,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (alive) {
                 tc_fence_after();
                 if (exact) {   // exact chunk: gauge move to r = mu_L, then V <- w V
-                    const float rho = g[kGScal + kSRho];
-                    float r[32];
-#pragma unroll 1
-                    for (int i = 0; i < DQK / 32; ++i) {
-                        tmem_ld32(tm + lane_base + C::TM_C + 32 * i, r);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) r[x] *= rho;
-                        tmem_st32(tm + lane_base + C::TM_C + 32 * i, r);
-                    }
-                    tmem_wait_st();
-                    scale_v_rows(sm + C::OFF_V + s * C::V_BYTES, g + kGW, st);
+                    exact_gauge_move_and_scale_v<C>(tm, lane_base, g[kGScal + kSRho], sm + C::OFF_V + s * C::V_BYTES,
+                                                    g + kGW, st);
                     fence_proxy_async_smem();
                     tc_fence_before();
                 }
@@ -672,31 +788,27 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (alive) {
                 const int len = min(kL, T - kL * c);
                 float *hc = hout + (size_t)kL * c * p.dv;
+                if (exact) {
+                    exact_epilogue<C>(tm, lane_base, coef_s + sb * kL, inv_s + sb * kL, hc, p.dv, len);
+                } else {
 #pragma unroll 1
-                for (int hh = 0; hh < 2; ++hh) {
-                    float rh[32], cf[32];
-                    tmem_ld32(tm + lane_base + C::TM_H + 32 * hh, rh);
-                    load32(coef_s + sb * kL + 32 * hh, cf);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int x = 0; x < 32; ++x) rh[x] *= cf[x];
-                    if (exact) {
-                        float ra[32];
-                        tmem_ld32(tm + lane_base + C::TM_S + 32 * hh, ra);
-                        load32(inv_s + sb * kL + 32 * hh, cf);
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float rh[32], cf[32];
+                        tmem_ld32(tm + lane_base + C::TM_H + 32 * hh, rh);
+                        load32(coef_s + sb * kL + 32 * hh, cf);
                         tmem_wait_ld();
 #pragma unroll
-                        for (int x = 0; x < 32; ++x) rh[x] = fmaf(ra[x], cf[x], rh[x]);
-                    }
-                    float *hrow = hc + (size_t)32 * hh * p.dv;
-                    const int n = min(32, len - 32 * hh);
-                    if (n == 32) {
+                        for (int x = 0; x < 32; ++x) rh[x] *= cf[x];
+                        float *hrow = hc + (size_t)32 * hh * p.dv;
+                        const int n = min(32, len - 32 * hh);
+                        if (n == 32) {
 #pragma unroll
-                        for (int x = 0; x < 32; ++x) hrow[(size_t)x * p.dv] = rh[x];
-                    } else {
+                            for (int x = 0; x < 32; ++x) hrow[(size_t)x * p.dv] = rh[x];
+                        } else {   // the last, partial chunk of a sequence
 #pragma unroll
-                        for (int x = 0; x < 32; ++x)
-                            if (x < n) hrow[(size_t)x * p.dv] = rh[x];
+                            for (int x = 0; x < 32; ++x)
+                                if (x < n) hrow[(size_t)x * p.dv] = rh[x];
+                        }
                     }
                 }
                 m_end = g[kGScal + kSMEnd];
@@ -736,122 +848,38 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
         const int trow = tk >> 1, half = tk & 1;     // n.q pass: token row, half of d_qk
         uint8_t *clo_s = sm + C::OFF_CLO;
-        named_barrier(3, 256);   // C_acc is initialised before either group splits it
         bool alive = true;
-        for (int c = 0; c < NC; ++c) {
+        // Chunk c-1 in the loop body below, then the operands of chunk c that need
+        // neither its split nor the P tile: V(c) <- w V(c) (fast chunks) and n.q_t.
+        // They overlap the readout MMAs of chunk c-1 instead of following them.
+        for (int c = -1; c < NC; ++c) {
+          if (c >= 0) {
             const int slot = c % kNG, s = c & 1, sb = c & 1;
             const float *g = gring + slot * C::G_FLOATS;
-            // the P tile, n.q / row-sum slots and the V stage of chunk c-2 are free
-            if (c >= 1) alive = alive && waitw(sh, &bar[B_H_FULL], (c - 1) & 1, kWhereTkH);
             alive = alive && waitw(sh, &bar[B_G_FULL + slot], (c / kNG) & 1, kWhereTkGate);
             const bool exact = alive && g[kGScal + kSExact] != 0.f;
-            // --- fast chunk: V <- w V in place, before the intra product
-            alive = alive && waitw(sh, &bar[B_KV_FULL + s], (c >> 1) & 1, kWhereTkKv);
-            if (alive && !exact) {
-                scale_v_rows(sm + C::OFF_V + s * C::V_BYTES, g + kGW, tk);
-                fence_proxy_async_smem();
-            }
-            named_barrier(2, 128);   // unconditional: every warp of the group takes every barrier
-            if (tk == 0 && alive && !exact) mbar_arrive(&bar[B_VT]);
             // --- upper half of the state split (its C_lo waits for the shared tile when d_qk = 256)
             if (c >= 1) alive = alive && waitw(sh, &bar[B_UPD_DONE], (c - 1) & 1, kWhereTkUpd);
             if (alive) {
                 tc_fence_after();
                 const bool mv = !exact && g[kGScal + kSRescale] != 0.f;
                 const float rho = g[kGScal + kSRho];
-#pragma unroll 1
-                for (int i = DQK / 64; i < DQK / 32; ++i)
-                    split_state_block<C>(tm, lane_base, i, mv, rho, C::BIG ? 2 : 0, clo_s, tk, 0);
+                split_range<C>(tm, lane_base, DQK / 64, DQK / 32, mv, rho, C::BIG ? 2 : 0, clo_s, tk, 0);
                 tmem_wait_st();
                 tc_fence_before();
             }
             named_barrier(2, 128);
             if (tk == 0 && alive) mbar_arrive(&bar[B_CONV0]);
-            // --- n.q_t in fp32 (coefficient AN_t = scale e^{b - mu_t})
-            alive = alive && waitw(sh, &bar[B_Q_FULL + s], (c >> 1) & 1, kWhereTkQ);
-            alive = alive && waitw(sh, &bar[B_N_READY + (c & 1)], (c >> 1) & 1, kWhereTkN);
-            if (alive) {
-                const uint8_t *Qs = sm + C::OFF_Q + s * C::Q_BYTES;
-                const float *nn = nbuf + (c & 1) * C::NBUF + (half ? 4 : 0);
-                float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                 make_float2(0.f, 0.f)};
-#pragma unroll 1
-                for (int g0 = 0; g0 < DQK / 16; g0 += 4) {
-                    uint4 u[4];
-                    float4 na[4], nb[4];
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        // the upper-half thread walks its chunks rotated by 4 so that the
-                        // pair of a token hits distinct banks
-                        const int ci = half ? (g0 + k4 + 4) % (DQK / 16) : g0 + k4;
-                        const int j = half * (DQK / 2) + 8 * ci;
-                        u[k4] = *reinterpret_cast<const uint4 *>(Qs + (j >> 6) * 8192 + sw128_offset(trow, (j & 63) >> 3));
-                        na[k4] = *reinterpret_cast<const float4 *>(nn + j);
-                        nb[k4] = *reinterpret_cast<const float4 *>(nn + j + 4);
-                    }
-#pragma unroll
-                    for (int k4 = 0; k4 < 4; ++k4) {
-                        acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].x), make_float2(na[k4].x, na[k4].y), acc[k4]);
-                        acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].y), make_float2(na[k4].z, na[k4].w), acc[k4]);
-                        acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].z), make_float2(nb[k4].x, nb[k4].y), acc[k4]);
-                        acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].w), make_float2(nb[k4].z, nb[k4].w), acc[k4]);
-                    }
-                }
-                float nq = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
-                nq += __shfl_xor_sync(0xffffffffu, nq, 1);
-                if (half == 0) nq_s[sb * kL + trow] = g[kGAN + trow] * nq;
-            }
-            named_barrier(2, 128);
-            if (tk == 0 && alive) {
-                mbar_arrive(&bar[B_Q_EMPTY + s]);
-                mbar_arrive(&bar[B_N_FREE + (c & 1)]);
-            }
+            // the P tile is free once PV(c-1) completed
+            if (c >= 1) alive = alive && waitw(sh, &bar[B_H_FULL], (c - 1) & 1, kWhereTkH);
             // --- P from S: lanes l and l+16 share token row 16 wq + (l & 15)
             alive = alive && waitw(sh, &bar[B_S_FULL], c & 1, kWhereTkS);
             if (alive) {
                 tc_fence_after();
-                float r0[32];   // lanes l and l + 16: columns [0, 32) and [32, 64) of row 16 wq + (l & 15)
-                tmem_ld16x2_32(tm + lane_base + C::TM_S, r0);
-                tmem_wait_ld();
-                const int t = 16 * wq + (lane & 15);
-                const int s0 = 32 * (lane >> 4);
-                float rs = 0.f;
-                if (exact) {
-                    const float mh = g[kGMh + t], ml = g[kGMl + t];
-                    float uh[32], ul[32];
-                    load32(g + kGUh + s0, uh);
-                    load32(g + kGUl + s0, ul);
-#pragma unroll
-                    for (int i = 0; i < 32; ++i) {
-                        const int sidx = s0 + i;
-                        const float e = (uh[i] - mh) + (ul[i] - ml);
-                        r0[i] = (sidx <= t) ? p.scale * r0[i] * exp2f(e) : 0.f;
-                        rs += r0[i];
-                    }
-                } else {
-                    float ww[32];
-                    load32(g + kGW + s0, ww);
-                    float2 r2 = make_float2(0.f, 0.f);
-#pragma unroll
-                    for (int i = 0; i < 32; i += 2) {
-                        r0[i] = (s0 + i <= t) ? r0[i] : 0.f;
-                        r0[i + 1] = (s0 + i + 1 <= t) ? r0[i + 1] : 0.f;
-                        r2 = __ffma2_rn(make_float2(r0[i], r0[i + 1]), make_float2(ww[i], ww[i + 1]), r2);
-                    }
-                    rs = r2.x + r2.y;
-                }
-#pragma unroll
-                for (int ch = 0; ch < 4; ++ch) {
-                    uint32_t hi[4], lo[4];
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) split_bf16x2(r0[8 * ch + 2 * i], r0[8 * ch + 2 * i + 1], hi[i], lo[i]);
-                    const int chunk = 4 * (lane >> 4) + ch;
-                    *reinterpret_cast<uint4 *>(Ps + sw128_offset(t, chunk)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                    *reinterpret_cast<uint4 *>(Ps + 8192 + sw128_offset(t, chunk)) =
-                        make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                }
-                rs += __shfl_xor_sync(0xffffffffu, rs, 16);
-                if (lane < 16) rs_s[sb * kL + t] = exact ? rs : g[kGAH + t] * rs;
+                if (exact)
+                    exact_p_pass(tm + lane_base + C::TM_S, g, Ps, rs_s + sb * kL, p.scale, wq, lane);
+                else
+                    p_pass(tm + lane_base + C::TM_S, g, Ps, rs_s + sb * kL, wq, lane);
                 tc_fence_before();
                 fence_proxy_async_smem();
             }
@@ -865,15 +893,72 @@ __global__ void __launch_bounds__(kThreads, 1)
                 alive = alive && waitw(sh, &bar[B_CLO_FREE], c & 1, kWhereTkClo);
                 if (alive) {
                     tc_fence_after();
-#pragma unroll 1
-                    for (int i = DQK / 64; i < DQK / 32; ++i)
-                        split_state_block<C>(tm, lane_base, i, false, 1.f, 3, clo_s, tk, 32 * i - DQK / 2);
+                    split_range<C>(tm, lane_base, DQK / 64, DQK / 32, false, 1.f, 3, clo_s, tk, 0);
                     fence_proxy_async_smem();
                     tc_fence_before();
                 }
                 named_barrier(2, 128);
                 if (tk == 0 && alive) mbar_arrive(&bar[B_CONV1]);
             }
+          }
+            if (c + 1 < NC) {
+                const int j = c + 1, sj = j & 1, slot_j = j % kNG;
+                const float *gj = gring + slot_j * C::G_FLOATS;
+                // the state group has read the n.q slot of chunk j-2 (its split of chunk c follows)
+                if (c >= 0) alive = alive && waitw(sh, &bar[B_CONV0], c & 1, kWhereTkConv);
+                alive = alive && waitw(sh, &bar[B_G_FULL + slot_j], (j / kNG) & 1, kWhereTkGate);
+                const bool ex = alive && gj[kGScal + kSExact] != 0.f;
+                // --- fast chunk: V <- w V in place, before the intra product
+                alive = alive && waitw(sh, &bar[B_KV_FULL + sj], (j >> 1) & 1, kWhereTkKv);
+                if (alive && !ex) {
+                    scale_v_rows(sm + C::OFF_V + sj * C::V_BYTES, gj + kGW, tk);
+                    fence_proxy_async_smem();
+                }
+                named_barrier(2, 128);   // unconditional: every warp of the group takes every barrier
+                if (tk == 0 && alive && !ex) mbar_arrive(&bar[B_VT]);
+                // --- n.q_t in fp32 (coefficient AN_t = scale e^{b - mu_t})
+                alive = alive && waitw(sh, &bar[B_Q_FULL + sj], (j >> 1) & 1, kWhereTkQ);
+                alive = alive && waitw(sh, &bar[B_N_READY + sj], (j >> 1) & 1, kWhereTkN);
+                if (alive) {
+                    const uint8_t *Qs = sm + C::OFF_Q + sj * C::Q_BYTES;
+                    const float *nn = nbuf + sj * C::NBUF + (half ? 4 : 0);
+                    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
+                                     make_float2(0.f, 0.f)};
+#pragma unroll 1
+                    for (int g0 = 0; g0 < DQK / 16; g0 += 4) {
+                        uint4 u[4];
+                        float4 na[4], nb[4];
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            // the upper-half thread walks its chunks rotated by 4 so that the
+                            // pair of a token hits distinct banks
+                            const int ci = half ? (g0 + k4 + 4) % (DQK / 16) : g0 + k4;
+                            const int jc = half * (DQK / 2) + 8 * ci;
+                            u[k4] = *reinterpret_cast<const uint4 *>(Qs + (jc >> 6) * 8192 +
+                                                                       sw128_offset(trow, (jc & 63) >> 3));
+                            na[k4] = *reinterpret_cast<const float4 *>(nn + jc);
+                            nb[k4] = *reinterpret_cast<const float4 *>(nn + jc + 4);
+                        }
+#pragma unroll
+                        for (int k4 = 0; k4 < 4; ++k4) {
+                            acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].x), make_float2(na[k4].x, na[k4].y), acc[k4]);
+                            acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].y), make_float2(na[k4].z, na[k4].w), acc[k4]);
+                            acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].z), make_float2(nb[k4].x, nb[k4].y), acc[k4]);
+                            acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].w), make_float2(nb[k4].z, nb[k4].w), acc[k4]);
+                        }
+                    }
+                    float nq = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
+                               ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+                    nq += __shfl_xor_sync(0xffffffffu, nq, 1);
+                    if (half == 0) nq_s[sj * kL + trow] = gj[kGAN + trow] * nq;
+                }
+                named_barrier(2, 128);
+                if (tk == 0 && alive) {
+                    mbar_arrive(&bar[B_Q_EMPTY + sj]);
+                    mbar_arrive(&bar[B_N_FREE + sj]);
+                }
+            }
+            if (c == -1) named_barrier(3, 256);   // C_acc is initialised before either group splits it
         }
     }
 
