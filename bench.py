@@ -76,7 +76,8 @@ def algorithmic(w, L=64):
 
 
 class ClockSampler:
-    """nvidia-smi clock/throttle samples taken while the timed region runs."""
+    """nvidia-smi clock/throttle samples; summary() keeps those that arrived while
+    the timed region ran (mark() brackets it)."""
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
@@ -84,13 +85,14 @@ class ClockSampler:
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.lines = []        # (arrival time, line)
+        self.window = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.t = threading.Thread(target=self._read, daemon=True)
             self.t.start()
@@ -101,7 +103,11 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.perf_counter(), line.strip()))
+
+    def mark(self, start: bool):
+        t = time.perf_counter()
+        self.window = (t, None) if start else (self.window[0], t)
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -115,7 +121,13 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        lines = self.lines
+        if self.window and self.window[1] is not None:
+            inside = [l for t, l in lines if self.window[0] <= t <= self.window[1] + 0.05]
+            lines = inside if inside else [l for _, l in lines]
+        else:
+            lines = [l for _, l in lines]
+        for line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 8:
                 continue
@@ -258,7 +270,7 @@ def run_reference(args, rank, world):
     w = inputs.WORKLOADS[args.workload]
     inp = make_inputs(w, n_decode_steps=32)
     # each step is a bounded sample so that the whole run stays within minutes
-    budget = max(2.0, min(args.ref_budget, 150.0 / max(1, args.steps)))
+    budget = max(0.5, min(args.ref_budget, 120.0 / max(1, args.steps)))
     vals = []
     cb = None
     for _ in range(max(1, args.steps)):
@@ -415,11 +427,13 @@ def run_ours(args, rank, world, local_rank):
     barrier()
     torch.cuda.synchronize(dev)
     with ClockSampler(local_rank if os.environ.get("CUDA_VISIBLE_DEVICES") is None else 0) as clk:
+        clk.mark(True)
         e0.record(stream)
         for i in range(args.steps):
             job.step(args.warmup + i)
         e1.record(stream)
         e1.synchronize()
+        clk.mark(False)
     torch.cuda.synchronize(dev)
     barrier()
     ms = slowest(e0.elapsed_time(e1) / args.steps)
@@ -500,7 +514,7 @@ def main():
     from xlstm_mlstm_matrix_b200.inputs import WORKLOADS
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=100)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", choices=[k for k in WORKLOADS if k != "tiny_fp32"],
