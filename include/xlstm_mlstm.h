@@ -194,7 +194,7 @@ XLSTM_API const char *xlstm_mlstm_version(void);
 
 /*
  * Which kernel xlstm_mlstm_fwd_chunkwise runs for desc: "tcgen05" (bf16
- * inputs, chunk 64, d_qk in {64, 128, 256}, d_v a multiple of 128), "simt"
+ * inputs, chunk 64, d_qk in {64, 128, 256}, d_v a multiple of 64), "simt"
  * (fp32 CUDA-core kernel: fp32 inputs and every other supported shape),
  * "copy" (T = 0) or "none" (invalid or unsupported desc).  Static storage.
  */

@@ -478,13 +478,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                         tma_prefetch_l2_3d(&tmk, 64 * b, kL * (c + 2), bh);
                         tma_prefetch_l2_3d(&tmq, 64 * b, kL * (c + 2), bh);
                     }
-                    for (int b = 0; b < 2; ++b) tma_prefetch_l2_3d(&tmv, v0 + 64 * b, kL * (c + 2), bh);
+                    for (int b = 0; b < 2; ++b)
+                        if (v0 + 64 * b < p.dv) tma_prefetch_l2_3d(&tmv, v0 + 64 * b, kL * (c + 2), bh);
                 }
                 if (c >= 2 && !wait1(sh, &bar[B_KV_EMPTY + s], ((c >> 1) - 1) & 1, kWhereTmaKvEmpty)) break;
                 mbar_arrive_expect_tx(&bar[B_KV_FULL + s], C::K_BYTES + C::V_BYTES);
                 uint8_t *Ks = sm + C::OFF_K + s * C::K_BYTES;
                 uint8_t *Vs = sm + C::OFF_V + s * C::V_BYTES;
                 for (int b = 0; b < C::NKB; ++b) tma_load_3d(Ks + b * 8192, &tmk, &bar[B_KV_FULL + s], 64 * b, kL * c, bh);
+                // a box past d_v (the upper half of a 64-row last slice) is zero-filled by the copy
                 for (int b = 0; b < 2; ++b) tma_load_3d(Vs + b * 8192, &tmv, &bar[B_KV_FULL + s], v0 + 64 * b, kL * c, bh);
                 ++kv_issued[s];
                 if (c >= 2 && !wait1(sh, &bar[B_Q_EMPTY + s], ((c >> 1) - 1) & 1, kWhereTmaQEmpty)) break;
@@ -730,11 +732,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int wq = warp - 4;             // TMEM lane quarter
         const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
         const int v = v0 + st;
+        const bool vok = v < p.dv;       // rows past d_v (a 64-row last slice) are computed on zeros and not stored
         float *hout = p.h + (size_t)bh * T * p.dv + v;
         uint8_t *clo_s = sm + C::OFF_CLO;
         {   // initial state: C_acc = C0 (gauge b = m = m0) or zero
             float r[32];
-            const float *src = p.C0 ? p.C0 + ((size_t)bh * p.dv + v) * DQK : nullptr;
+            const float *src = p.C0 && vok ? p.C0 + ((size_t)bh * p.dv + v) * DQK : nullptr;
 #pragma unroll 1
             for (int i = 0; i < DQK / 32; ++i) {
 #pragma unroll
@@ -788,9 +791,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (alive) {
                 const int len = min(kL, T - kL * c);
                 float *hc = hout + (size_t)kL * c * p.dv;
-                if (exact) {
+                if (exact && vok) {
                     exact_epilogue<C>(tm, lane_base, coef_s + sb * kL, inv_s + sb * kL, hc, p.dv, len);
-                } else {
+                } else if (vok) {
 #pragma unroll 1
                     for (int hh = 0; hh < 2; ++hh) {
                         float rh[32], cf[32];
@@ -825,7 +828,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         alive = alive && waitw(sh, &bar[B_UPD_DONE], (NC - 1) & 1, kWhereStFinal);
         if (alive) {
             tc_fence_after();
-            if (p.C1) {
+            if (p.C1 && vok) {
                 float r[32];
                 float *dst = p.C1 + ((size_t)bh * p.dv + v) * DQK;
 #pragma unroll 1
@@ -978,7 +981,7 @@ cudaError_t launch_dqk(const FwdArgs &a, cudaStream_t s, int fault) {
         !make_tmap_3d_bf16(&tv, a.v, a.dv, a.T, BH, 64, 64))
         return cudaErrorInvalidValue;
     TcParams p;
-    p.T = a.T; p.dv = a.dv; p.nslices = a.dv / kDvs; p.scale = a.scale;
+    p.T = a.T; p.dv = a.dv; p.nslices = (a.dv + kDvs - 1) / kDvs; p.scale = a.scale;
     p.ig = a.ig; p.fg = a.fg; p.C0 = a.C0; p.n0 = a.n0; p.m0 = a.m0;
     p.h = a.h; p.C1 = a.C1; p.n1 = a.n1; p.m1 = a.m1; p.status = a.status; p.fault = fault;
     auto kern = chunk_tc_kernel<DQK>;
@@ -992,7 +995,7 @@ cudaError_t launch_dqk(const FwdArgs &a, cudaStream_t s, int fault) {
 
 bool chunkwise_tc_supported(const FwdArgs &a) {
     if (a.dtype != XLSTM_BF16 || a.chunk != kL || a.T < 1) return false;
-    if (a.dv % kDvs != 0) return false;
+    if (a.dv % 64 != 0) return false;   // whole 64-row boxes; a last slice may hold 64 rows of 128
     if (a.dqk != 64 && a.dqk != 128 && a.dqk != 256) return false;
     return encode_tiled_fn() != nullptr;
 }
