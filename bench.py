@@ -304,7 +304,10 @@ class _Sequence:
                      torch.empty(w.B, w.H, w.d_qk, device=dev), torch.empty(w.B, w.H, device=dev)]
         self.desc = capi.make_desc(w.B, w.H, w.T, w.d_qk, w.d_v,
                                    capi.XLSTM_BF16 if bf else capi.XLSTM_F32, inp["qk_scale"], 64)
-        wsb = capi.xlstm_mlstm_workspace_size(self.desc)
+        # a workspace large enough for the segment-parallel path: a long sequence with few
+        # heads then runs as segment summaries, their combination and the chunkwise kernel
+        wsb = capi.xlstm_mlstm_workspace_size_parallel(self.desc)
+        segmented = wsb > capi.xlstm_mlstm_workspace_size(self.desc)
         self.ws = torch.zeros(wsb, device=dev, dtype=torch.uint8)
         self.fn = capi.load().xlstm_mlstm_fwd_chunkwise
         import ctypes
@@ -312,7 +315,8 @@ class _Sequence:
         self.argv = (ctypes.byref(self.desc), *(P(t) for t in self.ins), *(P(t) for t in self.outs),
                      P(self.ws), wsb, ctypes.c_void_p(stream.cuda_stream))
         self.stream = stream
-        self.kernel = "chunkwise"
+        self.kernel = "chunkwise (segment summaries + combine + chunkwise)" if segmented else "chunkwise"
+        self.launches = 3 if segmented else 1   # kernels per call
         self.name = "xlstm_mlstm_fwd_chunkwise"
 
     def step(self, i):
@@ -363,6 +367,7 @@ class _Decode:
         self.cs = ctypes.c_void_p(stream.cuda_stream)
         self.stream = stream
         self.kernel = "step"
+        self.launches = 1
         self.name = "xlstm_mlstm_step"
 
     def step(self, i, src=None):
@@ -500,7 +505,7 @@ def run_ours(args, rank, world, local_rank):
                          "peak_source": peak_src, "kernel": job.kernel,
                          "algorithmic_bytes_per_launch": bytes_, "flops_per_launch": flops,
                          "tensor_frac": flops / (ms * 1e-3) / 1e12 / bf16_peak},
-            "gpu_launches": args.steps,
+            "gpu_launches": args.steps * job.launches,
             "e2e": e2e,
             "clocks": clk.summary(),
             "kernel_source_sha": src_sha,

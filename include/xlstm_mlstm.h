@@ -98,7 +98,9 @@ typedef struct {
  *                      written, with C~ and n~ in that gauge.
  *   workspace        : device scratch of >= xlstm_mlstm_workspace_size(desc)
  *                      bytes, 256-byte aligned; its first 16 bytes are the
- *                      status block.  Calls sharing a workspace must not
+ *                      status block.  With >= xlstm_mlstm_workspace_size_parallel
+ *                      (desc) bytes a long sequence with few heads runs as
+ *                      parallel segments.  Calls sharing a workspace must not
  *                      overlap on the device.
  * Chunk lengths: 0 (= 64), 16, 32, 64; others return XLSTM_ERR_UNSUPPORTED.
  * Outputs must not overlap inputs.  T = 0 copies the state through.
@@ -176,6 +178,26 @@ XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise_noalloc(
 /* Workspace bytes xlstm_mlstm_fwd_chunkwise needs for desc (>= 256), or 0 for
  * a NULL desc. */
 XLSTM_API size_t xlstm_mlstm_workspace_size(const xlstm_mlstm_desc_t *desc);
+
+/*
+ * Workspace bytes with which xlstm_mlstm_fwd_chunkwise may run a long sequence
+ * as parallel segments (>= xlstm_mlstm_workspace_size(desc); equal to it when
+ * desc gains nothing from segments), or 0 for a NULL desc.
+ *
+ * The recurrence over a stretch of tokens is an affine map of the state (xLSTM
+ * page, "mLSTM (matrix LSTM)" eq. 1-3, with the stabilizer of the "sLSTM"
+ * section), so when B*H leaves most of the GPU idle (the tensor-core kernel's
+ * shapes only: bf16, chunk 64) the sequence is cut into segments of whole
+ * chunks: each segment but the last is first summarised from a zero state, the
+ * summaries are chained into every segment's entry state, and then all
+ * segments run at once.  The extra memory is about
+ * (segments - 1) * B * H * (d_v * d_qk + d_qk + 4) * 4 bytes; the extra traffic
+ * is one more read of k, v and the gates.  Results agree with the sequential
+ * evaluation to within rounding (the final state keeps the canonical m).
+ * With a smaller workspace (>= xlstm_mlstm_workspace_size) the call runs the
+ * sequence in one piece, as before.
+ */
+XLSTM_API size_t xlstm_mlstm_workspace_size_parallel(const xlstm_mlstm_desc_t *desc);
 
 /*
  * Reads the workspace status block written by the device: waits for `stream`,

@@ -19,7 +19,9 @@ def to_dev(x, dtype: str):
     return t.to(torch.bfloat16) if dtype == "bf16" else t
 
 
-def gpu_sequence(inp: dict, kind: str, chunk: int = 0, qk_scale=None, state=None):
+def gpu_sequence(inp: dict, kind: str, chunk: int = 0, qk_scale=None, state=None, parallel=False):
+    """The CUDA path through the C ABI.  parallel=True gives the chunkwise call a
+    workspace large enough for the segment-parallel evaluation."""
     w = inputs_workload(inp)
     dt = w.dtype
     q, k, v = (to_dev(inp[n], dt) for n in ("q", "k", "v"))
@@ -32,13 +34,22 @@ def gpu_sequence(inp: dict, kind: str, chunk: int = 0, qk_scale=None, state=None
         B, H, T, dqk = q.shape
         desc = capi.make_desc(B, H, T, dqk, v.shape[-1], capi.XLSTM_BF16 if dt == "bf16" else capi.XLSTM_F32,
                               scale, chunk)
-        ws = torch.zeros(max(256, capi.xlstm_mlstm_workspace_size(desc)), device=q.device, dtype=torch.uint8)
+        size = (capi.xlstm_mlstm_workspace_size_parallel if parallel else capi.xlstm_mlstm_workspace_size)(desc)
+        ws = torch.zeros(max(256, size), device=q.device, dtype=torch.uint8)
     h, (C, n, m) = capi.fwd(q, k, v, ig, fg, state=state, qk_scale=scale, chunk=chunk, kind=kind, workspace=ws)
     torch.cuda.synchronize()
     if ws is not None:   # no bounded device wait gave up
         code, where = capi.xlstm_mlstm_workspace_status(ws)
         assert code == capi.XLSTM_OK, f"device status {capi.xlstm_status_string(code)} (wait {where})"
     return h.cpu().numpy(), C.cpu().numpy(), n.cpu().numpy(), m.cpu().numpy()
+
+
+def small_inputs(B, H, T, dqk, dv, dtype, state, seed=7, gate="std", mean_i=0.0, std_i=1.5):
+    """Seeded inputs of the tiny workload's distributions at another shape."""
+    w = inputs.WORKLOADS["tiny_fp32"].replace(
+        B=B, H=H, T=T, d_qk=dqk, d_v=dv, dtype=dtype, gate=gate, mean_i=mean_i, std_i=std_i,
+        state="normal_m_uniform" if state else "zero", seed=seed)
+    return inputs.make_sequence(w)
 
 
 def inputs_workload(inp):

@@ -50,6 +50,37 @@ def test_workspace_size(lib):
     assert capi.xlstm_mlstm_workspace_size(d) >= 256
 
 
+def _seg_bytes(BH, G, dqk, dv):
+    """Scratch of G segments: (G-1) summaries per sequence, each region 256-aligned."""
+    a = lambda x: (x + 255) // 256 * 256
+    n = (G - 1) * BH
+    off_m = a(n * 16)
+    off_n = a(off_m + n * 4)
+    off_c = a(off_n + n * dqk * 4)
+    return a(off_c + n * dv * dqk * 4)
+
+
+def test_parallel_workspace_size(lib):
+    base = capi.xlstm_mlstm_workspace_size
+    par = capi.xlstm_mlstm_workspace_size_parallel
+    # long-context layer: 8 sequences of 1024 chunks on 148 SMs -> 18 segments of 57 chunks
+    d = capi.make_desc(1, 8, 65536, 128, 128, capi.XLSTM_BF16, 128 ** -0.5, 64)
+    assert par(d) == base(d) + _seg_bytes(8, 18, 128, 128)
+    # 2 heads x 4 value slices, 18 chunks: 2 segments of 9 chunks
+    d = capi.make_desc(1, 2, 1100, 256, 512, capi.XLSTM_BF16, 1.0, 64)
+    assert par(d) == base(d) + _seg_bytes(2, 2, 256, 512)
+    # no segments: enough heads to fill the GPU, too short, fp32, another chunk length
+    for B, H, T, dqk, dv, dt, L in [(8, 8, 4096, 256, 512, capi.XLSTM_BF16, 64),
+                                    (256, 4, 512, 64, 64, capi.XLSTM_BF16, 64),
+                                    (1, 1, 64 * 15, 128, 128, capi.XLSTM_BF16, 64),
+                                    (1, 8, 65536, 128, 128, capi.XLSTM_F32, 64),
+                                    (1, 8, 65536, 128, 128, capi.XLSTM_BF16, 32),
+                                    (1, 8, 65536, 96, 128, capi.XLSTM_BF16, 64)]:
+        d = capi.make_desc(B, H, T, dqk, dv, dt, 1.0, L)
+        assert par(d) == base(d), (B, H, T, dqk, dv, dt, L)
+    assert lib.xlstm_mlstm_workspace_size_parallel(None) == 0
+
+
 FAKE = dict(q=0x10000, k=0x20000, v=0x30000, i=0x40000, f=0x50000, h=0x60000, ws=0x100000)
 
 

@@ -11,7 +11,8 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_helpers import compare, fp32_row_tolerance, gpu_sequence, oracle_sequence, select_heads, to_dev
+from gpu_helpers import (compare, fp32_row_tolerance, gpu_sequence, oracle_sequence, select_heads, small_inputs,
+                         to_dev)
 import oracle
 from xlstm_mlstm_matrix_b200 import capi, inputs
 
@@ -43,13 +44,6 @@ SMALL = [  # B, H, T, dqk, dv
     (3, 2, 71, 256, 320),
 ]
 TC_SHAPES = [sh for sh in SMALL if sh[3] in (64, 128, 256) and sh[4] % 64 == 0]
-
-
-def small_inputs(B, H, T, dqk, dv, dtype, state, seed=7, gate="std", mean_i=0.0, std_i=1.5):
-    w = inputs.WORKLOADS["tiny_fp32"].replace(
-        B=B, H=H, T=T, d_qk=dqk, d_v=dv, dtype=dtype, gate=gate, mean_i=mean_i, std_i=std_i,
-        state="normal_m_uniform" if state else "zero", seed=seed)
-    return inputs.make_sequence(w)
 
 
 @pytest.mark.parametrize("kind", ["chunkwise", "recurrent"])

@@ -21,7 +21,7 @@ XLSTM_F32, XLSTM_BF16 = 0, 1
 EXPORTED = ("xlstm_mlstm_fwd_chunkwise", "xlstm_mlstm_fwd_recurrent", "xlstm_mlstm_step",
             "xlstm_mlstm_workspace_size", "xlstm_mlstm_workspace_status", "xlstm_status_string",
             "xlstm_mlstm_version", "xlstm_mlstm_chunkwise_kernel", "xlstm_mlstm_test_timeout_next",
-            "xlstm_mlstm_fwd_chunkwise_noalloc")
+            "xlstm_mlstm_fwd_chunkwise_noalloc", "xlstm_mlstm_workspace_size_parallel")
 
 
 class xlstm_mlstm_desc_t(ctypes.Structure):
@@ -59,6 +59,8 @@ def load(path: str = LIB_PATH):
     lib.xlstm_mlstm_step.restype = st
     lib.xlstm_mlstm_workspace_size.argtypes = [dp]
     lib.xlstm_mlstm_workspace_size.restype = sz
+    lib.xlstm_mlstm_workspace_size_parallel.argtypes = [dp]
+    lib.xlstm_mlstm_workspace_size_parallel.restype = sz
     lib.xlstm_mlstm_workspace_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
     lib.xlstm_mlstm_workspace_status.restype = st
     lib.xlstm_status_string.argtypes = [st]
@@ -133,6 +135,10 @@ def xlstm_mlstm_workspace_size(desc) -> int:
     return int(load().xlstm_mlstm_workspace_size(ctypes.byref(desc)))
 
 
+def xlstm_mlstm_workspace_size_parallel(desc) -> int:
+    return int(load().xlstm_mlstm_workspace_size_parallel(ctypes.byref(desc)))
+
+
 def xlstm_mlstm_workspace_status(workspace, stream=None):
     where = ctypes.c_int32(0)
     st = load().xlstm_mlstm_workspace_status(_p(workspace), ctypes.byref(where), _s(stream))
@@ -178,10 +184,12 @@ def _dtype_code(t):
 
 
 def fwd(q, k, v, i_pre, f_pre, state=None, qk_scale=None, chunk=0, kind="chunkwise",
-        stream=None, workspace=None, out=None):
+        stream=None, workspace=None, out=None, parallel=True):
     """Sequence forward through the C ABI.  q, k [B,H,T,dqk], v [B,H,T,dv]
     (bf16 or fp32, CUDA, contiguous), i_pre/f_pre [B,H,T] fp32; state is None
-    or (C [B,H,dv,dqk], n [B,H,dqk], m [B,H]).  Returns (h, (C, n, m))."""
+    or (C [B,H,dv,dqk], n [B,H,dqk], m [B,H]).  Returns (h, (C, n, m)).
+    Without a given workspace, the chunkwise call gets one large enough for the
+    segment-parallel evaluation of long sequences (parallel=False: the minimum)."""
     import torch
     B, H, T, dqk = q.shape
     dv = v.shape[-1]
@@ -199,8 +207,8 @@ def fwd(q, k, v, i_pre, f_pre, state=None, qk_scale=None, chunk=0, kind="chunkwi
     stream = stream if stream is not None else torch.cuda.current_stream(dev)
     if kind == "chunkwise":
         if workspace is None:
-            workspace = torch.empty(max(256, xlstm_mlstm_workspace_size(desc)), device=dev,
-                                    dtype=torch.uint8)
+            need = (xlstm_mlstm_workspace_size_parallel if parallel else xlstm_mlstm_workspace_size)(desc)
+            workspace = torch.empty(max(256, need), device=dev, dtype=torch.uint8)
         st = xlstm_mlstm_fwd_chunkwise(desc, q, k, v, i_pre, f_pre, C0, n0, m0, h, C1, n1, m1,
                                        workspace, workspace.numel(), stream)
     elif kind == "recurrent":

@@ -71,7 +71,7 @@ FwdArgs pack(const xlstm_mlstm_desc_t *d, const void *q, const void *k, const vo
     a.B = d->B; a.H = d->H; a.T = d->T; a.dqk = d->d_qk; a.dv = d->d_v;
     a.dtype = d->qkv_dtype; a.scale = d->qk_scale; a.chunk = d->chunk ? d->chunk : 64;
     a.q = q; a.k = k; a.v = v; a.ig = ig; a.fg = fg; a.C0 = C0; a.n0 = n0; a.m0 = m0;
-    a.h = h; a.C1 = C1; a.n1 = n1; a.m1 = m1; a.status = nullptr;
+    a.h = h; a.C1 = C1; a.n1 = n1; a.m1 = m1; a.status = nullptr; a.seg_ws = nullptr;
     return a;
 }
 
@@ -96,6 +96,15 @@ size_t xlstm_mlstm_workspace_size(const xlstm_mlstm_desc_t *desc) {
     return desc ? kWorkspaceBytes : 0;
 }
 
+size_t xlstm_mlstm_workspace_size_parallel(const xlstm_mlstm_desc_t *desc) {
+    if (!desc) return 0;
+    if (!dims_ok(desc)) return kWorkspaceBytes;
+    const FwdArgs a = pack(desc, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                           nullptr, nullptr, nullptr);
+    const xlstm::SegPlan sp = xlstm::segment_plan(a);
+    return kWorkspaceBytes + (sp.nseg > 1 ? sp.bytes : 0);
+}
+
 xlstm_status_t xlstm_mlstm_fwd_chunkwise(const xlstm_mlstm_desc_t *desc, const void *q,
                                          const void *k, const void *v, const float *i_pre,
                                          const float *f_pre, const float *C_in, const float *n_in,
@@ -113,6 +122,12 @@ xlstm_status_t xlstm_mlstm_fwd_chunkwise(const xlstm_mlstm_desc_t *desc, const v
     a.status = static_cast<int32_t *>(workspace);
     if (cudaMemsetAsync(workspace, 0, 16, stream) != cudaSuccess) return XLSTM_ERR_CUDA;
     if (a.T == 0) return pass_state_through(a, stream);
+    if (xlstm::chunkwise_tc_supported(a)) {
+        // a long sequence with few heads runs in parallel segments when the workspace holds their summaries
+        const xlstm::SegPlan sp = xlstm::segment_plan(a);
+        if (sp.nseg > 1 && workspace_bytes >= kWorkspaceBytes + sp.bytes)
+            a.seg_ws = static_cast<char *>(workspace) + kWorkspaceBytes;
+    }
     cudaError_t e = xlstm::chunkwise_tc_supported(a) ? xlstm::launch_chunkwise_tc(a, stream)
                                                      : xlstm::launch_chunkwise_simt(a, stream);
     return e == cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;

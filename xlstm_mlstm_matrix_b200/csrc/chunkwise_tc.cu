@@ -48,6 +48,7 @@
 
 #include "common.cuh"
 #include "sm100.cuh"
+#include "tc_common.cuh"
 #include "tma_host.cuh"
 
 namespace xlstm {
@@ -62,7 +63,6 @@ constexpr int kNG = 4;              // gate-ring slots
 constexpr double kRescale = 20.0;   // gauge drift allowed before the state is rescaled
 constexpr double kGrowth = 90.0;    // stabilizer rise inside a chunk handled by the fast path
 constexpr double kLog2e = 1.4426950408889634;
-constexpr uint64_t kTimeoutNs = 1000000000ull;   // 1 s per wait
 
 // Where a wait gave up (reported in the status block).
 enum : int32_t {
@@ -74,6 +74,7 @@ enum : int32_t {
 
 // Test hook: make the gate warp withhold one hand-off so that its consumers time out.
 int g_fault_next = 0;
+
 
 }  // namespace
 void set_chunkwise_tc_fault(int mode) { g_fault_next = mode; }
@@ -135,66 +136,32 @@ static_assert(B_COUNT <= 32, "barrier space");
 
 struct TcParams {
     int T, dv, nslices;
+    int nseg, seg_chunks, BH;   // the sequence in nseg segments of seg_chunks chunks (nseg = 1: whole)
     float scale;
     const float *ig, *fg, *C0, *n0, *m0;
+    const float *segC, *segN, *segM;   // entry states of segments 1 .. nseg-1
     float *h, *C1, *n1, *m1;
     int32_t *status;
     int fault;
 };
 
-struct Shared {
-    volatile int *abort_flag;
-    int32_t *status;
-};
-
-__device__ __forceinline__ void record_timeout(const Shared &sh, int where) {
-    *sh.abort_flag = 1;
-    if (sh.status && atomicCAS(&sh.status[kStatusCode], 0, (int32_t)XLSTM_ERR_TIMEOUT) == 0)
-        sh.status[kStatusWhere] = where;
+// Entry state of segment seg of sequence bh: the caller's (or none: zero state,
+// m = 0) for the first segment, the combined summaries of the earlier segments
+// for the others.  Pointers to the (bh) row: C [d_v][d_qk], n [d_qk], m scalar.
+template <int DQK>
+__device__ __forceinline__ const float *entry_C(const TcParams &p, int bh, int seg) {
+    if (seg == 0) return p.C0 ? p.C0 + (size_t)bh * p.dv * DQK : nullptr;
+    return p.segC + ((size_t)(seg - 1) * p.BH + bh) * p.dv * DQK;
 }
-
-// Single-thread bounded wait; gives up on timeout or when another role aborted.
-// Only the first test is inlined at the call sites; the waiting loop exists once.
-__device__ __noinline__ bool wait1_slow(const Shared &sh, uint64_t *bar, uint32_t parity, int where) {
-    const uint64_t t0 = global_timer_ns();
-    for (;;) {
-        // suspended in hardware (no issue slots) until the phase completes or 20 us pass
-        if (mbar_try_wait_suspend(bar, parity, 20000)) return true;
-        if (*sh.abort_flag) return false;
-        if (global_timer_ns() - t0 > kTimeoutNs) {
-            record_timeout(sh, where);
-            return false;
-        }
-    }
+template <int DQK>
+__device__ __forceinline__ const float *entry_n(const TcParams &p, int bh, int seg) {
+    if (seg == 0) return p.n0 ? p.n0 + (size_t)bh * DQK : nullptr;
+    return p.segN + ((size_t)(seg - 1) * p.BH + bh) * DQK;
 }
-__device__ __forceinline__ bool wait1(const Shared &sh, uint64_t *bar, uint32_t parity, int where) {
-    return mbar_try_wait(bar, parity) || wait1_slow(sh, bar, parity, where);
+__device__ __forceinline__ const float *entry_m(const TcParams &p, int bh, int seg) {
+    if (seg == 0) return p.m0 ? p.m0 + bh : nullptr;
+    return p.segM + (size_t)(seg - 1) * p.BH + bh;
 }
-// Whole-warp bounded wait: every lane agrees on the outcome.
-__device__ __forceinline__ bool waitw(const Shared &sh, uint64_t *bar, uint32_t parity, int where) {
-    return __all_sync(0xffffffffu, wait1(sh, bar, parity, where));
-}
-// Teardown wait: bounded, ignores the abort flag.
-__device__ __forceinline__ void drain_wait(uint64_t *bar, uint32_t parity) {
-    const uint64_t t0 = global_timer_ns();
-    while (!mbar_try_wait(bar, parity))
-        if (global_timer_ns() - t0 > kTimeoutNs) return;
-}
-
-__device__ __forceinline__ void unpack_bf16x8(const uint4 &u, float (&x)[8]) {
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        x[2 * i] = __uint_as_float(w[i] << 16);
-        x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-    }
-}
-__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-    return *reinterpret_cast<uint32_t *>(&v);
-}
-__device__ __forceinline__ float bf_lo(uint32_t u) { return __uint_as_float(u << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
 // (x0, x1) -> bf16 pairs hi = trunc(x), lo = round(x - hi): |x - hi - lo| <= 2^-16 |x|.
 // The high half is a plain truncation (two masks and a byte permute) so that
@@ -206,10 +173,6 @@ __device__ __forceinline__ void split_bf16x2(float x0, float x1, uint32_t &hi, u
                                                                 __uint_as_float((b & 0xFFFF0000u) ^ 0x80000000u)));
     lo = pack_bf16x2(r.x, r.y);
 }
-__device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u) {
-    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xFFFF0000u));
-}
-
 // Descriptor offsets (16-byte units) of K-step ks in a K-major 128B-swizzled tile of
 // 64-column boxes: boxes 8 KB apart for q / k tiles, 16 KB apart for the C_lo tile.
 __device__ __forceinline__ uint32_t kstep(int ks) { return (uint32_t)(((ks >> 2) * 8192 + (ks & 3) * 32) >> 4); }
@@ -223,30 +186,6 @@ __device__ __forceinline__ int nidx(int j) { return j + (j >= DQK / 2 ? 4 : 0); 
 __device__ __forceinline__ void split_double(double x, float &hi, float &lo) {
     hi = (float)x;
     lo = isfinite(hi) ? (float)(x - (double)hi) : 0.f;
-}
-
-// V <- w V in place: 1024 16-byte chunks of a 64-token x 128-value stage, chunk
-// e in row (token) (e mod 512) / 8; 128 threads, 8 chunks each.
-// All loads are issued before any store: the stores go to the same buffer, so
-// interleaving them would serialise every load behind the previous store.
-__device__ __forceinline__ void scale_v_rows(uint8_t *Vs, const float *w, int t128) {
-    uint4 u[8];
-    float ws[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int e = t128 + 128 * i;
-        u[i] = *reinterpret_cast<const uint4 *>(Vs + 16 * e);
-        ws[i] = w[(e & 511) >> 3];
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const float2 w2 = make_float2(ws[i], ws[i]);
-        const float2 a = __fmul2_rn(bf16x2_to_float2(u[i].x), w2), b = __fmul2_rn(bf16x2_to_float2(u[i].y), w2);
-        const float2 c = __fmul2_rn(bf16x2_to_float2(u[i].z), w2), d = __fmul2_rn(bf16x2_to_float2(u[i].w), w2);
-        u[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(b.x, b.y), pack_bf16x2(c.x, c.y), pack_bf16x2(d.x, d.y));
-    }
-#pragma unroll
-    for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4 *>(Vs + 16 * (t128 + 128 * i)) = u[i];
 }
 
 // 32 consecutive floats of a shared array into registers (broadcast loads).
@@ -436,11 +375,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *coef_s = inv_s + 2 * kL;                            // [2][64] AH_t/den_t
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int bh = blockIdx.x / p.nslices;
     const int slice = blockIdx.x % p.nslices;
+    const int seg = (blockIdx.x / p.nslices) % p.nseg;
+    const int bh = blockIdx.x / (p.nslices * p.nseg);
     const int v0 = slice * kDvs;
-    const int T = p.T;
+    const int t_base = kL * p.seg_chunks * seg;            // first token of this block's segment
+    const int T = min(p.T - t_base, kL * p.seg_chunks);    // tokens in the segment
     const int NC = (T + kL - 1) / kL;
+    const bool last_seg = seg == p.nseg - 1;               // the final state is written by the last segment
 
     if (tid == 0) {
         for (int i = 0; i < 2; ++i) {
@@ -475,24 +417,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const int s = c & 1;
                 if (c + 2 < NC) {   // chunk c+2 into L2 now, so that its stage load hits L2 later
                     for (int b = 0; b < C::NKB; ++b) {
-                        tma_prefetch_l2_3d(&tmk, 64 * b, kL * (c + 2), bh);
-                        tma_prefetch_l2_3d(&tmq, 64 * b, kL * (c + 2), bh);
+                        tma_prefetch_l2_3d(&tmk, 64 * b, t_base + kL * (c + 2), bh);
+                        tma_prefetch_l2_3d(&tmq, 64 * b, t_base + kL * (c + 2), bh);
                     }
                     for (int b = 0; b < 2; ++b)
-                        if (v0 + 64 * b < p.dv) tma_prefetch_l2_3d(&tmv, v0 + 64 * b, kL * (c + 2), bh);
+                        if (v0 + 64 * b < p.dv) tma_prefetch_l2_3d(&tmv, v0 + 64 * b, t_base + kL * (c + 2), bh);
                 }
                 if (c >= 2 && !wait1(sh, &bar[B_KV_EMPTY + s], ((c >> 1) - 1) & 1, kWhereTmaKvEmpty)) break;
                 mbar_arrive_expect_tx(&bar[B_KV_FULL + s], C::K_BYTES + C::V_BYTES);
                 uint8_t *Ks = sm + C::OFF_K + s * C::K_BYTES;
                 uint8_t *Vs = sm + C::OFF_V + s * C::V_BYTES;
-                for (int b = 0; b < C::NKB; ++b) tma_load_3d(Ks + b * 8192, &tmk, &bar[B_KV_FULL + s], 64 * b, kL * c, bh);
+                for (int b = 0; b < C::NKB; ++b) tma_load_3d(Ks + b * 8192, &tmk, &bar[B_KV_FULL + s], 64 * b, t_base + kL * c, bh);
                 // a box past d_v (the upper half of a 64-row last slice) is zero-filled by the copy
-                for (int b = 0; b < 2; ++b) tma_load_3d(Vs + b * 8192, &tmv, &bar[B_KV_FULL + s], v0 + 64 * b, kL * c, bh);
+                for (int b = 0; b < 2; ++b) tma_load_3d(Vs + b * 8192, &tmv, &bar[B_KV_FULL + s], v0 + 64 * b, t_base + kL * c, bh);
                 ++kv_issued[s];
                 if (c >= 2 && !wait1(sh, &bar[B_Q_EMPTY + s], ((c >> 1) - 1) & 1, kWhereTmaQEmpty)) break;
                 mbar_arrive_expect_tx(&bar[B_Q_FULL + s], C::Q_BYTES);
                 uint8_t *Qs = sm + C::OFF_Q + s * C::Q_BYTES;
-                for (int b = 0; b < C::NKB; ++b) tma_load_3d(Qs + b * 8192, &tmq, &bar[B_Q_FULL + s], 64 * b, kL * c, bh);
+                for (int b = 0; b < C::NKB; ++b) tma_load_3d(Qs + b * 8192, &tmq, &bar[B_Q_FULL + s], 64 * b, t_base + kL * c, bh);
                 ++q_issued[s];
             }
             // drain: every issued copy must land before shared memory is released
@@ -601,9 +543,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
     } else if (warp == 2) {
         // ===================== gate scan (float64) =====================
-        double m = p.m0 ? (double)p.m0[bh] : 0.0;
+        const float *m0 = entry_m(p, bh, seg);
+        double m = m0 ? (double)*m0 : 0.0;
         double b = m;
-        const float *ig = p.ig + (size_t)bh * T, *fg = p.fg + (size_t)bh * T;
+        const float *ig = p.ig + (size_t)bh * p.T + t_base, *fg = p.fg + (size_t)bh * p.T + t_base;
         for (int c = 0; c < NC; ++c) {
             const int slot = c % kNG;
             if (c >= kNG && !waitw(sh, &bar[B_G_EMPTY + slot], ((c / kNG) - 1) & 1, kWhereGateEmpty)) break;
@@ -670,8 +613,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         constexpr int NPL = DQK / 32;             // columns per lane
         const int j0 = lane * NPL;
         float nacc[NPL];
+        const float *n0 = entry_n<DQK>(p, bh, seg);
 #pragma unroll
-        for (int i = 0; i < NPL; ++i) nacc[i] = p.n0 ? p.n0[(size_t)bh * DQK + j0 + i] : 0.f;
+        for (int i = 0; i < NPL; ++i) nacc[i] = n0 ? n0[j0 + i] : 0.f;
 #pragma unroll
         for (int i = 0; i < NPL; ++i) nbuf[nidx<DQK>(j0 + i)] = nacc[i];
         __syncwarp();
@@ -722,7 +666,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&bar[B_G_EMPTY + slot]);
             }
         }
-        if (alive && slice == 0 && p.n1) {
+        if (alive && slice == 0 && last_seg && p.n1) {
 #pragma unroll
             for (int i = 0; i < NPL; ++i) p.n1[(size_t)bh * DQK + j0 + i] = nacc[i] * gsc;
         }
@@ -733,11 +677,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
         const int v = v0 + st;
         const bool vok = v < p.dv;       // rows past d_v (a 64-row last slice) are computed on zeros and not stored
-        float *hout = p.h + (size_t)bh * T * p.dv + v;
+        float *hout = p.h + ((size_t)bh * p.T + t_base) * p.dv + v;
         uint8_t *clo_s = sm + C::OFF_CLO;
         {   // initial state: C_acc = C0 (gauge b = m = m0) or zero
             float r[32];
-            const float *src = p.C0 && vok ? p.C0 + ((size_t)bh * p.dv + v) * DQK : nullptr;
+            const float *C0 = entry_C<DQK>(p, bh, seg);
+            const float *src = C0 && vok ? C0 + (size_t)v * DQK : nullptr;
 #pragma unroll 1
             for (int i = 0; i < DQK / 32; ++i) {
 #pragma unroll
@@ -748,7 +693,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         named_barrier(3, 256);   // C_acc is initialised before either group splits it
         bool alive = true;
-        float m_end = p.m0 ? p.m0[bh] : 0.f, gsc = 1.f;
+        const float *m0 = entry_m(p, bh, seg);
+        float m_end = m0 ? *m0 : 0.f, gsc = 1.f;
         for (int c = 0; c < NC; ++c) {
             const int slot = c % kNG, s = c & 1, sb = c & 1;
             const float *g = gring + slot * C::G_FLOATS;
@@ -828,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         alive = alive && waitw(sh, &bar[B_UPD_DONE], (NC - 1) & 1, kWhereStFinal);
         if (alive) {
             tc_fence_after();
-            if (p.C1 && vok) {
+            if (p.C1 && vok && last_seg) {
                 float r[32];
                 float *dst = p.C1 + ((size_t)bh * p.dv + v) * DQK;
 #pragma unroll 1
@@ -841,7 +787,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             make_float4(r[x] * gsc, r[x + 1] * gsc, r[x + 2] * gsc, r[x + 3] * gsc);
                 }
             }
-            if (slice == 0 && st == 0 && p.m1) p.m1[bh] = m_end;
+            if (slice == 0 && st == 0 && last_seg && p.m1) p.m1[bh] = m_end;
         }
         tc_fence_before();
     } else {
@@ -857,7 +803,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // They overlap the readout MMAs of chunk c-1 instead of following them.
         for (int c = -1; c < NC; ++c) {
           if (c >= 0) {
-            const int slot = c % kNG, s = c & 1, sb = c & 1;
+            const int slot = c % kNG, sb = c & 1;
             const float *g = gring + slot * C::G_FLOATS;
             alive = alive && waitw(sh, &bar[B_G_FULL + slot], (c / kNG) & 1, kWhereTkGate);
             const bool exact = alive && g[kGScal + kSExact] != 0.f;
@@ -984,21 +930,36 @@ cudaError_t launch_dqk(const FwdArgs &a, cudaStream_t s, int fault) {
     p.T = a.T; p.dv = a.dv; p.nslices = (a.dv + kDvs - 1) / kDvs; p.scale = a.scale;
     p.ig = a.ig; p.fg = a.fg; p.C0 = a.C0; p.n0 = a.n0; p.m0 = a.m0;
     p.h = a.h; p.C1 = a.C1; p.n1 = a.n1; p.m1 = a.m1; p.status = a.status; p.fault = fault;
+    p.BH = BH; p.nseg = 1; p.seg_chunks = (a.T + kL - 1) / kL;
+    p.segC = p.segN = p.segM = nullptr;
+    cudaError_t e;
+    if (a.seg_ws) {   // entry states of the segments first, on the same stream
+        const SegPlan sp = segment_plan(a);
+        if (sp.nseg > 1) {
+            if ((e = launch_segment_entry_states(a, sp, s)) != cudaSuccess) return e;
+            const char *ws = static_cast<const char *>(a.seg_ws);
+            p.nseg = sp.nseg; p.seg_chunks = sp.seg_chunks;
+            p.segC = reinterpret_cast<const float *>(ws + sp.off_C);
+            p.segN = reinterpret_cast<const float *>(ws + sp.off_N);
+            p.segM = reinterpret_cast<const float *>(ws + sp.off_M);
+        }
+    }
     auto kern = chunk_tc_kernel<DQK>;
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    kern<<<BH * p.nslices, kThreads, C::SMEM, s>>>(tq, tk, tv, p);
+    kern<<<BH * p.nseg * p.nslices, kThreads, C::SMEM, s>>>(tq, tk, tv, p);
     return cudaGetLastError();
 }
 
 }  // namespace
 
-bool chunkwise_tc_supported(const FwdArgs &a) {
+bool chunkwise_tc_shape_ok(const FwdArgs &a) {
     if (a.dtype != XLSTM_BF16 || a.chunk != kL || a.T < 1) return false;
     if (a.dv % 64 != 0) return false;   // whole 64-row boxes; a last slice may hold 64 rows of 128
-    if (a.dqk != 64 && a.dqk != 128 && a.dqk != 256) return false;
-    return encode_tiled_fn() != nullptr;
+    return a.dqk == 64 || a.dqk == 128 || a.dqk == 256;
 }
+
+bool chunkwise_tc_supported(const FwdArgs &a) { return chunkwise_tc_shape_ok(a) && encode_tiled_fn() != nullptr; }
 
 cudaError_t launch_chunkwise_tc(const FwdArgs &a, cudaStream_t s) {
     const int fault = g_fault_next;

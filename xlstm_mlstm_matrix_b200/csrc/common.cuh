@@ -19,7 +19,18 @@ struct FwdArgs {
     const float *C0, *n0, *m0;   // all null = zero state
     float *h, *C1, *n1, *m1;     // state outs may be null
     int32_t *status;             // device status block (4 x int32), may be null
+    void *seg_ws;                // scratch for the segment-parallel chunkwise path (null: sequential)
 };
+
+// How a long sequence is cut into segments that run in parallel (nseg = 1: not
+// cut), and where the segment summaries sit in the scratch (byte offsets).
+struct SegPlan {
+    int nseg = 1, seg_chunks = 0;
+    size_t off_S = 0, off_M = 0, off_N = 0, off_C = 0, bytes = 0;
+};
+SegPlan segment_plan(const FwdArgs &a);
+// Summaries of segments 0 .. nseg-2 and the entry states of segments 1 .. nseg-1.
+cudaError_t launch_segment_entry_states(const FwdArgs &a, const SegPlan &sp, cudaStream_t s);
 
 // Device status block layout (first 16 bytes of the workspace).
 enum : int32_t { kStatusCode = 0, kStatusWhere = 1 };
@@ -27,7 +38,8 @@ enum : int32_t { kStatusCode = 0, kStatusWhere = 1 };
 cudaError_t launch_step(const FwdArgs &a, cudaStream_t s);
 cudaError_t launch_recurrent(const FwdArgs &a, cudaStream_t s);
 cudaError_t launch_chunkwise_simt(const FwdArgs &a, cudaStream_t s);
-bool chunkwise_tc_supported(const FwdArgs &a);
+bool chunkwise_tc_shape_ok(const FwdArgs &a);     // shapes the tensor-core kernel takes
+bool chunkwise_tc_supported(const FwdArgs &a);    // ... and the driver's TMA encoder is available
 cudaError_t launch_chunkwise_tc(const FwdArgs &a, cudaStream_t s);
 void set_chunkwise_tc_fault(int mode);   // test hook: applies to the next launch only
 

@@ -1,0 +1,443 @@
+// Segment-parallel chunkwise forward, for long sequences with too few heads to
+// fill the GPU.
+//
+// The mLSTM recurrence (xLSTM page, "mLSTM (matrix LSTM)" eq. 1-3, with the
+// stabilizer of the "sLSTM" section) maps the state entering a stretch of tokens
+// to the state leaving it by an affine map whose coefficients depend only on the
+// stretch's own tokens.  A sequence cut into segments therefore runs in three
+// launches:
+//  1. summary (tensor cores), for every segment but the last, from a zero state:
+//     with F_t = sum_{r<=t} f~_r counted from the segment start, u_t = i~_t - F_t,
+//     F = F_last and u* = max_t u_t,
+//        C_seg = sum_t e^{u_t - u*} v_t k_t^T,   n_seg = sum_t e^{u_t - u*} k_t,
+//     the stabilized state the segment alone leaves, in the gauge m_seg = F + u*
+//     (the unrolled rule m_t = max(f~_t + m_{t-1}, i~_t) started from -inf);
+//  2. combine (CUDA cores): entry state of segment g+1 from that of g,
+//        m' = max(F + m, m_seg),
+//        C' = e^{F + m - m'} C + e^{m_seg - m'} C_seg    (n likewise);
+//     every coefficient is <= 1;
+//  3. the chunkwise kernel runs all segments at once, each from its entry state;
+//     the last one writes the final state.
+// Steps 1 and 2 read k, v and the gates once more and pass d_v x d_qk floats per
+// segment through the workspace; the sequential chain per block becomes nseg
+// times shorter.
+#include <math.h>
+
+#include <algorithm>
+
+#include "common.cuh"
+#include "sm100.cuh"
+#include "tc_common.cuh"
+#include "tma_host.cuh"
+
+namespace xlstm {
+namespace {
+
+using namespace sm100;
+
+constexpr int kL = 64;            // chunk length (tokens)
+constexpr int kDvs = 128;         // value rows per block
+constexpr int kSumThreads = 256;
+constexpr int kStages = 4;        // k / v stages in flight
+constexpr int kRing = 4;          // weight-ring slots
+constexpr int kMinSegChunks = 8;  // shortest segment worth a summary
+constexpr int kCombineThreads = 256;
+
+template <int DQK>
+struct SumCfg {
+    static constexpr int NKB = DQK / 64;          // 64-column boxes of k
+    static constexpr int K_BYTES = NKB * 8192;
+    static constexpr int V_BYTES = 2 * 8192;      // 128 value columns
+    static constexpr int OFF_K = 0;
+    static constexpr int OFF_V = OFF_K + kStages * K_BYTES;
+    static constexpr int OFF_W = OFF_V + kStages * V_BYTES;   // kRing x 64 weights
+    static constexpr int OFF_RED = OFF_W + kRing * kL * 4;    // 8 warps x (F, u*) doubles
+    static constexpr int OFF_BAR = OFF_RED + 8 * 16;
+    static constexpr int NBARS = 24;
+    static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
+    static constexpr int SMEM = OFF_MISC + 64 + 1024;         // + alignment slack
+    static_assert(SMEM <= 232448, "shared memory budget");
+};
+
+enum : int {
+    S_KV_FULL = 0, S_KV_EMPTY = S_KV_FULL + kStages, S_VS = S_KV_EMPTY + kStages, S_W_FULL = S_VS + kStages,
+    S_W_EMPTY = S_W_FULL + kRing, S_DONE = S_W_EMPTY + kRing, S_DRAIN, S_COUNT
+};
+static_assert(S_COUNT <= 24, "barrier space");
+
+// Where a wait of the summary kernel gave up (status block; the chunkwise
+// kernel's codes are below 40).
+enum : int32_t { kWhereSumKvEmpty = 41, kWhereSumVs, kWhereSumWEmpty, kWhereSumKv, kWhereSumW, kWhereSumDone };
+
+struct SumParams {
+    int T, dv, nslices, nsum, seg_chunks, BH;   // nsum = nseg - 1 summaries per sequence
+    const float *ig, *fg;
+    float *segC, *segN;   // [nsum][BH][d_v][d_qk], [nsum][BH][d_qk]
+    double *segS;         // [nsum][BH][2]: F, m_seg
+    int32_t *status;
+};
+
+// Inclusive prefix sum over the 64 tokens of a chunk held two per lane (a, b):
+// returns the sum before token a (within the chunk) and the chunk total.
+__device__ __forceinline__ void chunk_scan(double fa, double fb, double &excl, double &total) {
+    double incl = fa + fb;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const double y = __shfl_up_sync(0xffffffffu, incl, o);
+        if ((threadIdx.x & 31) >= o) incl += y;
+    }
+    excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if ((threadIdx.x & 31) == 0) excl = 0.0;
+    total = __shfl_sync(0xffffffffu, incl, 31);
+}
+
+// Per segment: its state from a zero start (C_seg, n_seg) and the scalars F, m_seg.
+// Block = (sequence, segment, 128 value rows); warps: 0 TMA, 1 MMA (owns TMEM),
+// 2 weights, 3 n_seg, 4-7 w V in place and the read-out of C_seg.
+template <int DQK>
+__global__ void __launch_bounds__(kSumThreads, 1)
+    seg_summary_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
+                       const SumParams p) {
+    using C = SumCfg<DQK>;
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    uint64_t *bar = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(sm + C::OFF_MISC);
+    Shared sh{reinterpret_cast<volatile int *>(sm + C::OFF_MISC + 4), p.status};
+    float *wring = reinterpret_cast<float *>(sm + C::OFF_W);
+    double *red = reinterpret_cast<double *>(sm + C::OFF_RED);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int slice = blockIdx.x % p.nslices;
+    const int g = (blockIdx.x / p.nslices) % p.nsum;
+    const int bh = blockIdx.x / (p.nslices * p.nsum);
+    const int v0 = slice * kDvs;
+    const int NC = p.seg_chunks;   // a summarised segment is never the last: all its chunks are full
+    const int t_base = kL * NC * g;
+    const float *ig = p.ig + (size_t)bh * p.T + t_base, *fg = p.fg + (size_t)bh * p.T + t_base;
+
+    if (tid == 0) {
+        for (int i = 0; i < kStages; ++i) {
+            mbar_init(&bar[S_KV_FULL + i], 1);
+            mbar_init(&bar[S_KV_EMPTY + i], 2);   // the update MMAs and the n_seg warp read k
+            mbar_init(&bar[S_VS + i], 1);
+        }
+        for (int i = 0; i < kRing; ++i) {
+            mbar_init(&bar[S_W_FULL + i], 1);
+            mbar_init(&bar[S_W_EMPTY + i], 2);    // the w V group and the n_seg warp read w
+        }
+        mbar_init(&bar[S_DONE], 1);
+        mbar_init(&bar[S_DRAIN], 1);
+        *sh.abort_flag = 0;
+        fence_mbar_init();
+        tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmv);
+    }
+    if (warp == 1) {
+        tmem_alloc(tmem_slot, DQK);
+        tmem_relinquish();
+    }
+    // F and u* of the segment: warp w scans a contiguous run of chunks, with F
+    // counted from the run's start; the runs are then joined in order.
+    {
+        const int per = (NC + 7) / 8;
+        const int c0 = warp * per, c1 = min(NC, c0 + per);
+        double frun = 0.0, umax = -INFINITY;
+        for (int c = c0; c < c1; ++c) {
+            const int t = kL * c + 2 * lane;
+            const double fa = fg[t], fb = fg[t + 1], ia = ig[t], ib = ig[t + 1];
+            double excl, total;
+            chunk_scan(fa, fb, excl, total);
+            const double Fa = frun + excl + fa, Fb = Fa + fb;
+            umax = fmax(umax, fmax(ia - Fa, ib - Fb));
+            frun += total;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) umax = fmax(umax, __shfl_xor_sync(0xffffffffu, umax, o));
+        if (lane == 0) { red[2 * warp] = frun; red[2 * warp + 1] = umax; }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *tmem_slot;
+    double Fseg = 0.0, ustar = -INFINITY;
+    for (int w = 0; w < 8; ++w) {
+        ustar = fmax(ustar, red[2 * w + 1] - Fseg);
+        Fseg += red[2 * w];
+    }
+
+    if (warp == 0) {
+        // ===================== TMA producer =====================
+        if (lane == 0) {
+            int issued[kStages] = {};
+            for (int c = 0; c < NC; ++c) {
+                const int s = c % kStages;
+                if (c >= kStages && !wait1(sh, &bar[S_KV_EMPTY + s], ((c / kStages) - 1) & 1, kWhereSumKvEmpty)) break;
+                mbar_arrive_expect_tx(&bar[S_KV_FULL + s], C::K_BYTES + C::V_BYTES);
+                uint8_t *Ks = sm + C::OFF_K + s * C::K_BYTES;
+                uint8_t *Vs = sm + C::OFF_V + s * C::V_BYTES;
+                for (int b = 0; b < C::NKB; ++b)
+                    tma_load_3d(Ks + b * 8192, &tmk, &bar[S_KV_FULL + s], 64 * b, t_base + kL * c, bh);
+                // a box past d_v (the upper half of a 64-row last slice) is zero-filled by the copy
+                for (int b = 0; b < 2; ++b)
+                    tma_load_3d(Vs + b * 8192, &tmv, &bar[S_KV_FULL + s], v0 + 64 * b, t_base + kL * c, bh);
+                ++issued[s];
+            }
+            for (int s = 0; s < kStages; ++s)   // every issued copy lands before shared memory is released
+                if (issued[s]) drain_wait(&bar[S_KV_FULL + s], (issued[s] - 1) & 1);
+        }
+    } else if (warp == 1) {
+        // ===================== MMA issuer: C_seg += (w V)^T K =====================
+        if (lane == 0) {
+            const uint32_t idU = make_idesc(128, DQK, kFmtBF16, kFmtBF16, 1, 1);
+            bool issued = false;
+            for (int c = 0; c < NC; ++c) {
+                const int s = c % kStages;
+                if (!wait1(sh, &bar[S_VS + s], (c / kStages) & 1, kWhereSumVs)) break;
+                tc_fence_after();
+                const uint64_t dv_mn = smem_desc_sw128(smem_u32(sm + C::OFF_V + s * C::V_BYTES), 8192, 1024);
+                const uint64_t dk_mn = smem_desc_sw128(smem_u32(sm + C::OFF_K + s * C::K_BYTES), 8192, 1024);
+#pragma unroll 1
+                for (int ks = 0; ks < kL / 16; ++ks)
+                    mma_f16_ss(tm, dv_mn + (uint32_t)(ks * 2048 >> 4), dk_mn + (uint32_t)(ks * 2048 >> 4), idU,
+                               (c > 0 || ks > 0) ? 1u : 0u);
+                issued = true;
+                tc_commit(&bar[S_KV_EMPTY + s]);
+            }
+            if (issued) {   // C_seg complete, and nothing in flight when tensor memory is freed
+                tc_commit(&bar[S_DONE]);
+                tc_commit(&bar[S_DRAIN]);
+                drain_wait(&bar[S_DRAIN], 0);
+            }
+        }
+    } else if (warp == 2) {
+        // ===================== weights w_t = e^{u_t - u*} =====================
+        double frun = 0.0;
+        for (int c = 0; c < NC; ++c) {
+            const int slot = c % kRing;
+            if (c >= kRing && !waitw(sh, &bar[S_W_EMPTY + slot], ((c / kRing) - 1) & 1, kWhereSumWEmpty)) break;
+            const int t = kL * c + 2 * lane;
+            const double fa = fg[t], fb = fg[t + 1], ia = ig[t], ib = ig[t + 1];
+            double excl, total;
+            chunk_scan(fa, fb, excl, total);
+            const double Fa = frun + excl + fa, Fb = Fa + fb;
+            float *w = wring + slot * kL;
+            w[2 * lane] = expf((float)(ia - Fa - ustar));
+            w[2 * lane + 1] = expf((float)(ib - Fb - ustar));
+            frun += total;
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&bar[S_W_FULL + slot]);
+        }
+        if (lane == 0 && slice == 0) {
+            double *sc = p.segS + ((size_t)g * p.BH + bh) * 2;
+            sc[0] = Fseg;
+            sc[1] = Fseg + ustar;
+        }
+    } else if (warp == 3) {
+        // ===================== n_seg = sum_t w_t k_t =====================
+        constexpr int NPL = DQK / 32;   // columns per lane
+        const int j0 = lane * NPL;
+        const uint32_t box = j0 >> 6, chk = (j0 & 63) >> 3, within = (j0 & 7) * 2;
+        float nacc[NPL];
+#pragma unroll
+        for (int i = 0; i < NPL; ++i) nacc[i] = 0.f;
+        bool alive = true;
+        for (int c = 0; c < NC; ++c) {
+            const int s = c % kStages, slot = c % kRing;
+            alive = waitw(sh, &bar[S_KV_FULL + s], (c / kStages) & 1, kWhereSumKv) &&
+                    waitw(sh, &bar[S_W_FULL + slot], (c / kRing) & 1, kWhereSumW);
+            if (!alive) break;
+            const uint8_t *Ks = sm + C::OFF_K + s * C::K_BYTES + box * 8192 + within;
+            const float *w = wring + slot * kL;
+#pragma unroll 4
+            for (int t = 0; t < kL; ++t) {
+                const uint8_t *src = Ks + sw128_offset(t, chk);
+                const float wt = w[t];
+                if (NPL == 8) {
+                    float x[8];
+                    unpack_bf16x8(*reinterpret_cast<const uint4 *>(src), x);
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) nacc[i % NPL] = fmaf(wt, x[i], nacc[i % NPL]);
+                } else if (NPL == 4) {
+                    const uint2 u = *reinterpret_cast<const uint2 *>(src);
+                    const float x[4] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y)};
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) nacc[i % NPL] = fmaf(wt, x[i], nacc[i % NPL]);
+                } else {
+                    const uint32_t u = *reinterpret_cast<const uint32_t *>(src);
+                    const float x[2] = {bf_lo(u), bf_hi(u)};
+#pragma unroll
+                    for (int i = 0; i < 2; ++i) nacc[i % NPL] = fmaf(wt, x[i], nacc[i % NPL]);
+                }
+            }
+            __syncwarp();
+            if (lane == 0) {
+                mbar_arrive(&bar[S_KV_EMPTY + s]);
+                mbar_arrive(&bar[S_W_EMPTY + slot]);
+            }
+        }
+        if (alive && slice == 0) {
+            float *dst = p.segN + ((size_t)g * p.BH + bh) * DQK + j0;
+#pragma unroll
+            for (int i = 0; i < NPL; ++i) dst[i] = nacc[i];
+        }
+    } else {
+        // ===================== w V in place; read-out of C_seg =====================
+        const int t128 = tid - 128;
+        bool alive = true;
+        for (int c = 0; c < NC; ++c) {
+            const int s = c % kStages, slot = c % kRing;
+            alive = alive && waitw(sh, &bar[S_KV_FULL + s], (c / kStages) & 1, kWhereSumKv) &&
+                    waitw(sh, &bar[S_W_FULL + slot], (c / kRing) & 1, kWhereSumW);
+            if (alive) {
+                scale_v_rows(sm + C::OFF_V + s * C::V_BYTES, wring + slot * kL, t128);
+                fence_proxy_async_smem();   // the MMA (async proxy) reads what these stores wrote
+            }
+            // unconditional: every warp of the group takes every barrier, even after
+            // another warp of it gave up
+            named_barrier(1, 128);
+            if (t128 == 0 && alive) {
+                mbar_arrive(&bar[S_VS + s]);
+                mbar_arrive(&bar[S_W_EMPTY + slot]);
+            }
+        }
+        alive = alive && waitw(sh, &bar[S_DONE], 0, kWhereSumDone);
+        const int v = v0 + t128;
+        if (alive && v < p.dv) {   // warp-uniform: d_v is a multiple of 64
+            tc_fence_after();
+            const uint32_t lane_base = (uint32_t)(32 * (warp - 4)) << 16;
+            float *dst = p.segC + (((size_t)g * p.BH + bh) * p.dv + v) * DQK;
+            float r[32];
+#pragma unroll 1
+            for (int i = 0; i < DQK / 32; ++i) {
+                tmem_ld32(tm + lane_base + 32 * i, r);
+                tmem_wait_ld();
+#pragma unroll
+                for (int x = 0; x < 32; x += 4)
+                    *reinterpret_cast<float4 *>(dst + 32 * i + x) = make_float4(r[x], r[x + 1], r[x + 2], r[x + 3]);
+            }
+        }
+        tc_fence_before();
+    }
+
+    __syncthreads();
+    if (warp == 1) {
+        tc_fence_after();
+        tmem_dealloc(tm, DQK);
+    }
+}
+
+struct CombineParams {
+    int BH, dv, dqk, nsum;
+    const float *C0, *n0, *m0;   // caller's initial state (null: zero state, m = 0)
+    float *segC, *segN, *segM;   // summaries in, entry states of segments 1..nsum out (in place)
+    const double *segS;
+};
+
+// Entry states, in place over the summaries: slot g becomes the state entering
+// segment g+1.  One thread per 4 consecutive floats of (C, n) of one sequence;
+// every thread runs the scalar chain of gauges itself, in float64.
+__global__ void __launch_bounds__(kCombineThreads) seg_combine_kernel(const CombineParams p) {
+    const int bh = blockIdx.y;
+    const int nC4 = p.dv * p.dqk / 4, n4 = nC4 + p.dqk / 4;
+    const int e4 = blockIdx.x * kCombineThreads + threadIdx.x;
+    if (e4 >= n4) return;
+    const bool isC = e4 < nC4;
+    float4 x = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (isC && p.C0) x = reinterpret_cast<const float4 *>(p.C0 + (size_t)bh * p.dv * p.dqk)[e4];
+    if (!isC && p.n0) x = reinterpret_cast<const float4 *>(p.n0 + (size_t)bh * p.dqk)[e4 - nC4];
+    double m = p.m0 ? (double)p.m0[bh] : 0.0;
+    for (int g = 0; g < p.nsum; ++g) {
+        const double F = p.segS[((size_t)g * p.BH + bh) * 2], ms = p.segS[((size_t)g * p.BH + bh) * 2 + 1];
+        // the new gauge, rounded to the fp32 m the chunkwise kernel reads, so that the
+        // state handed on is exactly in the gauge it is labelled with
+        const double mp = (double)(float)fmax(F + m, ms);
+        const float a = (float)exp(F + m - mp), b = (float)exp(ms - mp);
+        float4 *slot = isC ? reinterpret_cast<float4 *>(p.segC + ((size_t)g * p.BH + bh) * p.dv * p.dqk) + e4
+                           : reinterpret_cast<float4 *>(p.segN + ((size_t)g * p.BH + bh) * p.dqk) + (e4 - nC4);
+        const float4 y = *slot;
+        x = make_float4(fmaf(a, x.x, b * y.x), fmaf(a, x.y, b * y.y), fmaf(a, x.z, b * y.z), fmaf(a, x.w, b * y.w));
+        *slot = x;
+        if (e4 == 0) p.segM[(size_t)g * p.BH + bh] = (float)mp;
+        m = mp;
+    }
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0, v = 0;
+        n = (cudaGetDevice(&dev) == cudaSuccess &&
+             cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+                ? v
+                : 148;
+    }
+    return n;
+}
+
+template <int DQK>
+cudaError_t launch_summaries_dqk(const FwdArgs &a, const SegPlan &sp, cudaStream_t s) {
+    using C = SumCfg<DQK>;
+    const int BH = a.B * a.H;
+    CUtensorMap tk, tv;
+    if (!make_tmap_3d_bf16(&tk, a.k, DQK, a.T, BH, 64, 64) || !make_tmap_3d_bf16(&tv, a.v, a.dv, a.T, BH, 64, 64))
+        return cudaErrorInvalidValue;
+    char *ws = static_cast<char *>(a.seg_ws);
+    SumParams p;
+    p.T = a.T; p.dv = a.dv; p.nslices = (a.dv + kDvs - 1) / kDvs; p.nsum = sp.nseg - 1;
+    p.seg_chunks = sp.seg_chunks; p.BH = BH; p.ig = a.ig; p.fg = a.fg;
+    p.segC = reinterpret_cast<float *>(ws + sp.off_C);
+    p.segN = reinterpret_cast<float *>(ws + sp.off_N);
+    p.segS = reinterpret_cast<double *>(ws + sp.off_S);
+    p.status = a.status;
+    auto kern = seg_summary_kernel<DQK>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    kern<<<BH * p.nsum * p.nslices, kSumThreads, C::SMEM, s>>>(tk, tv, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    CombineParams q;
+    q.BH = BH; q.dv = a.dv; q.dqk = DQK; q.nsum = p.nsum;
+    q.C0 = a.C0; q.n0 = a.n0; q.m0 = a.m0;
+    q.segC = p.segC; q.segN = p.segN; q.segM = reinterpret_cast<float *>(ws + sp.off_M); q.segS = p.segS;
+    const int n4 = (a.dv * DQK + DQK) / 4;
+    seg_combine_kernel<<<dim3((n4 + kCombineThreads - 1) / kCombineThreads, BH), kCombineThreads, 0, s>>>(q);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+SegPlan segment_plan(const FwdArgs &a) {
+    SegPlan sp;
+    sp.nseg = 1;
+    if (!chunkwise_tc_shape_ok(a)) return sp;
+    const long long BH = (long long)a.B * a.H;
+    const long long blocks = BH * ((a.dv + kDvs - 1) / kDvs);
+    const int NC = (a.T + kL - 1) / kL;
+    const long long fit = sm_count() / blocks;   // segments per sequence that still fit one wave
+    int G = (int)std::min<long long>(fit, NC / kMinSegChunks);
+    if (G < 2) return sp;
+    sp.seg_chunks = (NC + G - 1) / G;
+    G = (NC + sp.seg_chunks - 1) / sp.seg_chunks;
+    if (G < 2) return sp;
+    sp.nseg = G;
+    const size_t nsum = (size_t)(G - 1) * BH;
+    sp.off_S = 0;
+    sp.off_M = align256(sp.off_S + nsum * 2 * sizeof(double));
+    sp.off_N = align256(sp.off_M + nsum * sizeof(float));
+    sp.off_C = align256(sp.off_N + nsum * a.dqk * sizeof(float));
+    sp.bytes = align256(sp.off_C + nsum * (size_t)a.dv * a.dqk * sizeof(float));
+    return sp;
+}
+
+cudaError_t launch_segment_entry_states(const FwdArgs &a, const SegPlan &sp, cudaStream_t s) {
+    switch (a.dqk) {
+        case 64: return launch_summaries_dqk<64>(a, sp, s);
+        case 128: return launch_summaries_dqk<128>(a, sp, s);
+        case 256: return launch_summaries_dqk<256>(a, sp, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+}  // namespace xlstm
