@@ -479,7 +479,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait1(sh, &bar[B_G_FULL + slot], (c / kNG) & 1, kWhereMmaGate)) break;
                 const bool exact = gring[slot * C::G_FLOATS + kGScal + kSExact] != 0.f;
                 if (!wait1(sh, &bar[B_CONV0], c & 1, kWhereMmaConv)) break;
-                if (!wait1(sh, &bar[B_OPS], c & 1, kWhereMmaOps)) break;
+                // w V(c) is waited here, not before the intra part: the token group's next
+                // phase of B_VT (chunk c+1) may complete during the readout, and a wait
+                // for the earlier phase after that would never return
                 if (!exact && !wait1(sh, &bar[B_VT], (nfast++) & 1, kWhereMmaVt)) break;
                 if (c >= 1 && !prev_exact && !wait1(sh, &bar[B_H_EMPTY], (c - 1) & 1, kWhereMmaHEmpty)) break;
                 tc_fence_after();
@@ -511,6 +513,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 // intra part: fast chunks accumulate (w V)^T (mask S)^T onto H; exact
                 // chunks put V^T P^T into the S columns
+                // P(c) is needed only from here: the C Q^T MMAs above overlap its computation
+                // (B_OPS cannot run a phase ahead: P(c+1) needs S(c+1), issued after this chunk)
+                if (!wait1(sh, &bar[B_OPS], c & 1, kWhereMmaOps)) break;
+                tc_fence_after();
                 {
                     const uint64_t dp = smem_desc_sw128(p_addr, 16, 1024);
                     const uint32_t dst = exact ? tm + C::TM_S : tm + C::TM_H;
