@@ -712,7 +712,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const bool mv = !exact && g[kGScal + kSRescale] != 0.f;
                 const float rho = g[kGScal + kSRho];
-                split_range<C>(tm, lane_base, 0, DQK / 64, mv, rho, C::BIG ? 1 : 0, clo_s, st, 0);
+                // d_qk = 256: the state group, which comes to the split from the previous
+                // epilogue, takes columns 0-63; the token group the other 192 (below)
+                split_range<C>(tm, lane_base, 0, C::BIG ? 2 : DQK / 64, mv, rho, C::BIG ? 1 : 0, clo_s, st, 0);
                 tmem_wait_st();
                 if (C::BIG) fence_proxy_async_smem();
                 tc_fence_before();
@@ -819,7 +821,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 tc_fence_after();
                 const bool mv = !exact && g[kGScal + kSRescale] != 0.f;
                 const float rho = g[kGScal + kSRho];
-                split_range<C>(tm, lane_base, DQK / 64, DQK / 32, mv, rho, C::BIG ? 2 : 0, clo_s, tk, 0);
+                if (C::BIG) {   // columns 64-127 with their C_lo (shared tile), then C_hi of 128-255
+                    split_range<C>(tm, lane_base, 2, 4, mv, rho, 1, clo_s, tk, 64);
+                    split_range<C>(tm, lane_base, 4, 8, mv, rho, 2, clo_s, tk, 0);
+                } else {
+                    split_range<C>(tm, lane_base, DQK / 64, DQK / 32, mv, rho, 0, clo_s, tk, 0);
+                }
                 tmem_wait_st();
                 tc_fence_before();
             }
