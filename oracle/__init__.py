@@ -46,6 +46,8 @@ def _declare(lib):
     lib.mlstm_oracle_forward.argtypes = [i64, i64, i64, i64, i64, dbl] + [ptr] * 12 + [cint]
     lib.mlstm_oracle_step.restype = cint
     lib.mlstm_oracle_step.argtypes = [i64, i64, i64, i64, dbl] + [ptr] * 12 + [cint]
+    lib.mlstm_oracle_output_gate.restype = cint
+    lib.mlstm_oracle_output_gate.argtypes = [i64, ptr, ptr, ptr]
     return lib
 
 
@@ -125,3 +127,15 @@ def step(q, k, v, i_pre, f_pre, C, n, m, qk_scale=1.0, threads: int | None = Non
     if rc != 0:
         raise RuntimeError(f"mlstm_oracle_step failed ({rc})")
     return h, C1, n1, m1
+
+
+def output_gate(h_tilde, o_pre, lib=None):
+    """h = sigmoid(o_pre) * h~, element by element (the page's eq. 3 output gate).
+    h_tilde and o_pre of one shape; returns float64 of that shape."""
+    h_tilde, o_pre = _f64(h_tilde), _f64(o_pre)
+    assert h_tilde.shape == o_pre.shape
+    h = np.empty(h_tilde.shape)
+    lib = lib or load_library()
+    if lib.mlstm_oracle_output_gate(h.size, _p(h_tilde), _p(o_pre), _p(h)) != 0:
+        raise RuntimeError("mlstm_oracle_output_gate failed")
+    return h

@@ -199,3 +199,18 @@ int mlstm_oracle_step(int64_t B, int64_t H, int64_t dqk, int64_t dv, double qk_s
     return mlstm_oracle_forward(B, H, 1, dqk, dv, qk_scale, q, k, v, ig, fg,
                                 C, n, m, h, C1, n1, m1, nthreads);
 }
+
+/*
+ * Output stage of the mLSTM (xLSTM page, "mLSTM (matrix LSTM)" eq. 3, and the
+ * o_t line of the page's forward_recurrent listing): h_t = o_t * h~_t with
+ * o_t the logistic sigmoid of the output-gate pre-activation, element by
+ * element.  count elements of h_tilde and o_pre; h may alias neither.
+ */
+int mlstm_oracle_output_gate(int64_t count, const double *h_tilde, const double *o_pre, double *h)
+{
+    if (count < 0 || (count > 0 && (!h_tilde || !o_pre || !h)))
+        return 1;
+    for (int64_t i = 0; i < count; ++i)
+        h[i] = h_tilde[i] / (1.0 + exp(-o_pre[i]));
+    return 0;
+}

@@ -310,6 +310,20 @@ def pin_p10_hand_case(lib):
                float(abs(m.ravel()[0] - g["m"][0])))
 
 
+def pin_p11_output_gate(lib):
+    """Closed forms of h = sigmoid(o) h~ (page eq. 3): o = 0 halves h~; o = ln 3
+    keeps three quarters; o and -o together give h~ back (sigmoid(o) +
+    sigmoid(-o) = 1); o = +40 passes h~ through, o = -40 shuts it (below e^-40)."""
+    rng = np.random.default_rng(11)
+    h = rng.normal(size=(3, 50)) * np.exp(rng.uniform(-20, 20, size=(3, 50)))
+    o = rng.normal(scale=3.0, size=h.shape)
+    g = lambda oo: oracle.output_gate(h, np.broadcast_to(oo, h.shape), lib=lib)
+    errs = [_rel(g(0.0), 0.5 * h), _rel(g(np.log(3.0)), 0.75 * h),
+            _rel(oracle.output_gate(h, o, lib=lib) + oracle.output_gate(h, -o, lib=lib), h),
+            _rel(g(40.0), h), float(np.max(np.abs(g(-40.0)) / np.abs(h))) * 1e-3]
+    return max(errs)
+
+
 PINS = [
     ("P1 quadratic form", pin_p1_quadratic, 1e-12),
     ("P2 unstabilized recurrence", pin_p2_unstabilized, 1e-10),
@@ -320,4 +334,5 @@ PINS = [
     ("P7 composition", pin_p7_composition, 1e-12),
     ("P8 gauge", pin_p8_gauge, 1e-12),
     ("P10 hand case", pin_p10_hand_case, 1e-14),
+    ("P11 output gate", pin_p11_output_gate, 1e-15),
 ]

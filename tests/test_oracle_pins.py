@@ -77,6 +77,8 @@ MUTANTS = {
     "stale stabilizer": ("m = m_new;\n    }", "}"),
     "normaliser without gate": ("j->n[c] = fp * j->n[c] + ip * kt[c]", "j->n[c] = fp * j->n[c] + kt[c]"),
     "input gate unstabilized": ("const double ip = exp(it - m_new);", "const double ip = exp(it);"),
+    "output gate sign": ("h_tilde[i] / (1.0 + exp(-o_pre[i]))", "h_tilde[i] / (1.0 + exp(o_pre[i]))"),
+    "output gate missing": ("h_tilde[i] / (1.0 + exp(-o_pre[i]))", "h_tilde[i]"),
 }
 
 

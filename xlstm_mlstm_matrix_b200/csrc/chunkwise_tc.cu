@@ -40,8 +40,8 @@
 //
 // Warps: 0 TMA producer (and L2 prefetch two chunks ahead), 1 MMA issuer (owns
 // TMEM), 2 gate scan, 3 normaliser,
-// 4-7 state group (lower half of the state split, epilogue), 8-11 token group
-// (w V, upper half of the state split, n.q, P).
+// 4-7 state group (the first columns of the state split, epilogue), 8-11 token
+// group (w V, the other columns of the state split, n.q, P).
 // Every wait is bounded: one that gives up records XLSTM_ERR_TIMEOUT in the
 // status block; each role drains what it has in flight, TMEM is freed, return.
 #include <math.h>
@@ -83,6 +83,10 @@ namespace {
 template <int DQK>
 struct Cfg {
     static constexpr bool BIG = DQK == 256;
+    // 32-column blocks of the state split done by the state group; the token group
+    // does the rest.  The state group comes to the split from the previous chunk's
+    // epilogue, the token group straight from the update, so it takes the larger part.
+    static constexpr int SPLIT_ST = BIG ? 2 : (DQK == 128 ? 1 : 0);
     static constexpr int NKB = DQK / 64;               // 64-column boxes of q and k
     static constexpr int Q_BYTES = NKB * 8192;
     static constexpr int K_BYTES = NKB * 8192;
@@ -707,14 +711,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c >= 1) alive = alive && waitw(sh, &bar[B_UPD_DONE], (c - 1) & 1, kWhereStUpd);
             alive = alive && waitw(sh, &bar[B_G_FULL + slot], (c / kNG) & 1, kWhereStGate);
             const bool exact = alive && g[kGScal + kSExact] != 0.f;
-            // --- lower half of the state split (C_lo of it: TMEM, or the shared tile)
+            // --- first columns of the state split (C_lo of it: TMEM, or the shared tile)
             if (alive) {
                 tc_fence_after();
                 const bool mv = !exact && g[kGScal + kSRescale] != 0.f;
                 const float rho = g[kGScal + kSRho];
-                // d_qk = 256: the state group, which comes to the split from the previous
-                // epilogue, takes columns 0-63; the token group the other 192 (below)
-                split_range<C>(tm, lane_base, 0, C::BIG ? 2 : DQK / 64, mv, rho, C::BIG ? 1 : 0, clo_s, st, 0);
+                // columns [0, 32 SPLIT_ST); the token group splits the rest
+                if (C::SPLIT_ST > 0)
+                    split_range<C>(tm, lane_base, 0, C::SPLIT_ST, mv, rho, C::BIG ? 1 : 0, clo_s, st, 0);
                 tmem_wait_st();
                 if (C::BIG) fence_proxy_async_smem();
                 tc_fence_before();
@@ -815,7 +819,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             const float *g = gring + slot * C::G_FLOATS;
             alive = alive && waitw(sh, &bar[B_G_FULL + slot], (c / kNG) & 1, kWhereTkGate);
             const bool exact = alive && g[kGScal + kSExact] != 0.f;
-            // --- upper half of the state split (its C_lo waits for the shared tile when d_qk = 256)
+            // --- the other columns of the state split (for d_qk = 256, the C_lo of columns
+            //     128-255 waits for the shared tile)
             if (c >= 1) alive = alive && waitw(sh, &bar[B_UPD_DONE], (c - 1) & 1, kWhereTkUpd);
             if (alive) {
                 tc_fence_after();
@@ -825,7 +830,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     split_range<C>(tm, lane_base, 2, 4, mv, rho, 1, clo_s, tk, 64);
                     split_range<C>(tm, lane_base, 4, 8, mv, rho, 2, clo_s, tk, 0);
                 } else {
-                    split_range<C>(tm, lane_base, DQK / 64, DQK / 32, mv, rho, 0, clo_s, tk, 0);
+                    split_range<C>(tm, lane_base, C::SPLIT_ST, DQK / 32, mv, rho, 0, clo_s, tk, 0);
                 }
                 tmem_wait_st();
                 tc_fence_before();

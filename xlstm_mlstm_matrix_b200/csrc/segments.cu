@@ -38,9 +38,9 @@ using namespace sm100;
 constexpr int kL = 64;            // chunk length (tokens)
 constexpr int kDvs = 128;         // value rows per block
 constexpr int kSumThreads = 256;
-constexpr int kStages = 4;        // k / v stages in flight
-constexpr int kRing = 4;          // weight-ring slots
+constexpr int kRing = 4;          // weight-ring slots (even: each slot has one producer warp)
 constexpr int kMinSegChunks = 8;  // shortest segment worth a summary
+constexpr int kMaxSegChunks = 1024;   // longest segment (its per-chunk F offsets sit in shared memory)
 constexpr int kCombineThreads = 256;
 
 template <int DQK>
@@ -48,22 +48,22 @@ struct SumCfg {
     static constexpr int NKB = DQK / 64;          // 64-column boxes of k
     static constexpr int K_BYTES = NKB * 8192;
     static constexpr int V_BYTES = 2 * 8192;      // 128 value columns
+    // k / v stages in flight: as many as ~190 KB hold (the copies are the bound)
+    static constexpr int STAGES = DQK == 256 ? 4 : (DQK == 128 ? 6 : 8);
     static constexpr int OFF_K = 0;
-    static constexpr int OFF_V = OFF_K + kStages * K_BYTES;
-    static constexpr int OFF_W = OFF_V + kStages * V_BYTES;   // kRing x 64 weights
+    static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
+    static constexpr int OFF_W = OFF_V + STAGES * V_BYTES;    // kRing x 64 weights
     static constexpr int OFF_RED = OFF_W + kRing * kL * 4;    // 8 warps x (F, u*) doubles
-    static constexpr int OFF_BAR = OFF_RED + 8 * 16;
-    static constexpr int NBARS = 24;
+    static constexpr int OFF_F = OFF_RED + 8 * 16;            // per-chunk F offsets (doubles)
+    static constexpr int OFF_BAR = OFF_F + kMaxSegChunks * 8;
+    // barriers: KV_FULL, KV_EMPTY, VS per stage; W_FULL, W_EMPTY per ring slot; DONE, DRAIN
+    static constexpr int B_KV_FULL = 0, B_KV_EMPTY = STAGES, B_VS = 2 * STAGES, B_W_FULL = 3 * STAGES,
+                         B_W_EMPTY = B_W_FULL + kRing, B_DONE = B_W_EMPTY + kRing, B_DRAIN = B_DONE + 1,
+                         NBARS = B_DRAIN + 1;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM = OFF_MISC + 64 + 1024;         // + alignment slack
     static_assert(SMEM <= 232448, "shared memory budget");
 };
-
-enum : int {
-    S_KV_FULL = 0, S_KV_EMPTY = S_KV_FULL + kStages, S_VS = S_KV_EMPTY + kStages, S_W_FULL = S_VS + kStages,
-    S_W_EMPTY = S_W_FULL + kRing, S_DONE = S_W_EMPTY + kRing, S_DRAIN, S_COUNT
-};
-static_assert(S_COUNT <= 24, "barrier space");
 
 // Where a wait of the summary kernel gave up (status block; the chunkwise
 // kernel's codes are below 40).
@@ -93,7 +93,7 @@ __device__ __forceinline__ void chunk_scan(double fa, double fb, double &excl, d
 
 // Per segment: its state from a zero start (C_seg, n_seg) and the scalars F, m_seg.
 // Block = (sequence, segment, 128 value rows); warps: 0 TMA, 1 MMA (owns TMEM),
-// 2 weights, 3 n_seg, 4-7 w V in place and the read-out of C_seg.
+// 2-3 weights, 4-7 w V in place, n_seg and the read-out of C_seg.
 template <int DQK>
 __global__ void __launch_bounds__(kSumThreads, 1)
     seg_summary_kernel(const __grid_constant__ CUtensorMap tmk, const __grid_constant__ CUtensorMap tmv,
@@ -106,6 +106,7 @@ __global__ void __launch_bounds__(kSumThreads, 1)
     Shared sh{reinterpret_cast<volatile int *>(sm + C::OFF_MISC + 4), p.status};
     float *wring = reinterpret_cast<float *>(sm + C::OFF_W);
     double *red = reinterpret_cast<double *>(sm + C::OFF_RED);
+    double *chunkF = reinterpret_cast<double *>(sm + C::OFF_F);   // F before chunk c, from its run's start
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int slice = blockIdx.x % p.nslices;
@@ -117,20 +118,29 @@ __global__ void __launch_bounds__(kSumThreads, 1)
     const float *ig = p.ig + (size_t)bh * p.T + t_base, *fg = p.fg + (size_t)bh * p.T + t_base;
 
     if (tid == 0) {
-        for (int i = 0; i < kStages; ++i) {
-            mbar_init(&bar[S_KV_FULL + i], 1);
-            mbar_init(&bar[S_KV_EMPTY + i], 2);   // the update MMAs and the n_seg warp read k
-            mbar_init(&bar[S_VS + i], 1);
+        for (int i = 0; i < C::STAGES; ++i) {
+            mbar_init(&bar[C::B_KV_FULL + i], 1);
+            mbar_init(&bar[C::B_KV_EMPTY + i], 2);   // the update MMAs and the n_seg sum read k
+            mbar_init(&bar[C::B_VS + i], 1);
         }
         for (int i = 0; i < kRing; ++i) {
-            mbar_init(&bar[S_W_FULL + i], 1);
-            mbar_init(&bar[S_W_EMPTY + i], 2);    // the w V group and the n_seg warp read w
+            mbar_init(&bar[C::B_W_FULL + i], 1);
+            mbar_init(&bar[C::B_W_EMPTY + i], 1);
         }
-        mbar_init(&bar[S_DONE], 1);
-        mbar_init(&bar[S_DRAIN], 1);
+        mbar_init(&bar[C::B_DONE], 1);
+        mbar_init(&bar[C::B_DRAIN], 1);
         *sh.abort_flag = 0;
         fence_mbar_init();
-        tma_prefetch_desc(&tmk); tma_prefetch_desc(&tmv);
+        // the first stages load while the gates are scanned
+        for (int c = 0; c < C::STAGES && c < NC; ++c) {
+            mbar_arrive_expect_tx(&bar[C::B_KV_FULL + c], C::K_BYTES + C::V_BYTES);
+            for (int b = 0; b < C::NKB; ++b)
+                tma_load_3d(sm + C::OFF_K + c * C::K_BYTES + b * 8192, &tmk, &bar[C::B_KV_FULL + c], 64 * b,
+                            t_base + kL * c, bh);
+            for (int b = 0; b < 2; ++b)
+                tma_load_3d(sm + C::OFF_V + c * C::V_BYTES + b * 8192, &tmv, &bar[C::B_KV_FULL + c], v0 + 64 * b,
+                            t_base + kL * c, bh);
+        }
     }
     if (warp == 1) {
         tmem_alloc(tmem_slot, DQK);
@@ -138,17 +148,26 @@ __global__ void __launch_bounds__(kSumThreads, 1)
     }
     // F and u* of the segment: warp w scans a contiguous run of chunks, with F
     // counted from the run's start; the runs are then joined in order.
+    const int per = (NC + 7) / 8;   // chunks per run
     {
-        const int per = (NC + 7) / 8;
         const int c0 = warp * per, c1 = min(NC, c0 + per);
         double frun = 0.0, umax = -INFINITY;
+        float fan = 0.f, fbn = 0.f, ian = 0.f, ibn = 0.f;   // the next chunk's gates, loaded ahead
+        if (c0 < c1) {
+            const int t = kL * c0 + 2 * lane;
+            fan = fg[t]; fbn = fg[t + 1]; ian = ig[t]; ibn = ig[t + 1];
+        }
         for (int c = c0; c < c1; ++c) {
-            const int t = kL * c + 2 * lane;
-            const double fa = fg[t], fb = fg[t + 1], ia = ig[t], ib = ig[t + 1];
+            const double fa = fan, fb = fbn, ia = ian, ib = ibn;
+            if (c + 1 < c1) {
+                const int t = kL * (c + 1) + 2 * lane;
+                fan = fg[t]; fbn = fg[t + 1]; ian = ig[t]; ibn = ig[t + 1];
+            }
             double excl, total;
             chunk_scan(fa, fb, excl, total);
             const double Fa = frun + excl + fa, Fb = Fa + fb;
             umax = fmax(umax, fmax(ia - Fa, ib - Fb));
+            if (lane == 0) chunkF[c] = frun;
             frun += total;
         }
 #pragma unroll
@@ -168,22 +187,23 @@ __global__ void __launch_bounds__(kSumThreads, 1)
     if (warp == 0) {
         // ===================== TMA producer =====================
         if (lane == 0) {
-            int issued[kStages] = {};
-            for (int c = 0; c < NC; ++c) {
-                const int s = c % kStages;
-                if (c >= kStages && !wait1(sh, &bar[S_KV_EMPTY + s], ((c / kStages) - 1) & 1, kWhereSumKvEmpty)) break;
-                mbar_arrive_expect_tx(&bar[S_KV_FULL + s], C::K_BYTES + C::V_BYTES);
+            int issued[C::STAGES] = {};
+            for (int c = 0; c < C::STAGES && c < NC; ++c) issued[c] = 1;   // issued before the gate scan
+            for (int c = C::STAGES; c < NC; ++c) {
+                const int s = c % C::STAGES;
+                if (!wait1(sh, &bar[C::B_KV_EMPTY + s], ((c / C::STAGES) - 1) & 1, kWhereSumKvEmpty)) break;
+                mbar_arrive_expect_tx(&bar[C::B_KV_FULL + s], C::K_BYTES + C::V_BYTES);
                 uint8_t *Ks = sm + C::OFF_K + s * C::K_BYTES;
                 uint8_t *Vs = sm + C::OFF_V + s * C::V_BYTES;
                 for (int b = 0; b < C::NKB; ++b)
-                    tma_load_3d(Ks + b * 8192, &tmk, &bar[S_KV_FULL + s], 64 * b, t_base + kL * c, bh);
+                    tma_load_3d(Ks + b * 8192, &tmk, &bar[C::B_KV_FULL + s], 64 * b, t_base + kL * c, bh);
                 // a box past d_v (the upper half of a 64-row last slice) is zero-filled by the copy
                 for (int b = 0; b < 2; ++b)
-                    tma_load_3d(Vs + b * 8192, &tmv, &bar[S_KV_FULL + s], v0 + 64 * b, t_base + kL * c, bh);
+                    tma_load_3d(Vs + b * 8192, &tmv, &bar[C::B_KV_FULL + s], v0 + 64 * b, t_base + kL * c, bh);
                 ++issued[s];
             }
-            for (int s = 0; s < kStages; ++s)   // every issued copy lands before shared memory is released
-                if (issued[s]) drain_wait(&bar[S_KV_FULL + s], (issued[s] - 1) & 1);
+            for (int s = 0; s < C::STAGES; ++s)   // every issued copy lands before shared memory is released
+                if (issued[s]) drain_wait(&bar[C::B_KV_FULL + s], (issued[s] - 1) & 1);
         }
     } else if (warp == 1) {
         // ===================== MMA issuer: C_seg += (w V)^T K =====================
@@ -191,8 +211,8 @@ __global__ void __launch_bounds__(kSumThreads, 1)
             const uint32_t idU = make_idesc(128, DQK, kFmtBF16, kFmtBF16, 1, 1);
             bool issued = false;
             for (int c = 0; c < NC; ++c) {
-                const int s = c % kStages;
-                if (!wait1(sh, &bar[S_VS + s], (c / kStages) & 1, kWhereSumVs)) break;
+                const int s = c % C::STAGES;
+                if (!wait1(sh, &bar[C::B_VS + s], (c / C::STAGES) & 1, kWhereSumVs)) break;
                 tc_fence_after();
                 const uint64_t dv_mn = smem_desc_sw128(smem_u32(sm + C::OFF_V + s * C::V_BYTES), 8192, 1024);
                 const uint64_t dk_mn = smem_desc_sw128(smem_u32(sm + C::OFF_K + s * C::K_BYTES), 8192, 1024);
@@ -201,106 +221,104 @@ __global__ void __launch_bounds__(kSumThreads, 1)
                     mma_f16_ss(tm, dv_mn + (uint32_t)(ks * 2048 >> 4), dk_mn + (uint32_t)(ks * 2048 >> 4), idU,
                                (c > 0 || ks > 0) ? 1u : 0u);
                 issued = true;
-                tc_commit(&bar[S_KV_EMPTY + s]);
+                tc_commit(&bar[C::B_KV_EMPTY + s]);
             }
             if (issued) {   // C_seg complete, and nothing in flight when tensor memory is freed
-                tc_commit(&bar[S_DONE]);
-                tc_commit(&bar[S_DRAIN]);
-                drain_wait(&bar[S_DRAIN], 0);
+                tc_commit(&bar[C::B_DONE]);
+                tc_commit(&bar[C::B_DRAIN]);
+                drain_wait(&bar[C::B_DRAIN], 0);
             }
         }
-    } else if (warp == 2) {
+    } else if (warp == 2 || warp == 3) {
         // ===================== weights w_t = e^{u_t - u*} =====================
-        double frun = 0.0;
-        for (int c = 0; c < NC; ++c) {
-            const int slot = c % kRing;
-            if (c >= kRing && !waitw(sh, &bar[S_W_EMPTY + slot], ((c / kRing) - 1) & 1, kWhereSumWEmpty)) break;
+        // Warp 2 takes the even chunks, warp 3 the odd ones (a ring slot always has
+        // the same producer); F at a chunk's start comes from the first pass.  The
+        // gates of a warp's next chunk are loaded while it processes the current one
+        // (scalar loads: a sequence's gates start at an arbitrary float offset).
+        int c = warp - 2;
+        float fan = 0.f, fbn = 0.f, ian = 0.f, ibn = 0.f;
+        if (c < NC) {
             const int t = kL * c + 2 * lane;
-            const double fa = fg[t], fb = fg[t + 1], ia = ig[t], ib = ig[t + 1];
+            fan = fg[t]; fbn = fg[t + 1]; ian = ig[t]; ibn = ig[t + 1];
+        }
+        for (; c < NC; c += 2) {
+            const int slot = c % kRing;
+            const double fa = fan, fb = fbn, ia = ian, ib = ibn;
+            if (c + 2 < NC) {
+                const int t = kL * (c + 2) + 2 * lane;
+                fan = fg[t]; fbn = fg[t + 1]; ian = ig[t]; ibn = ig[t + 1];
+            }
+            double F0 = chunkF[c];
+            for (int w = 0; w < c / per; ++w) F0 += red[2 * w];
+            if (c >= kRing && !waitw(sh, &bar[C::B_W_EMPTY + slot], ((c / kRing) - 1) & 1, kWhereSumWEmpty)) break;
             double excl, total;
             chunk_scan(fa, fb, excl, total);
-            const double Fa = frun + excl + fa, Fb = Fa + fb;
+            const double Fa = F0 + excl + fa, Fb = Fa + fb;
             float *w = wring + slot * kL;
             w[2 * lane] = expf((float)(ia - Fa - ustar));
             w[2 * lane + 1] = expf((float)(ib - Fb - ustar));
-            frun += total;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&bar[S_W_FULL + slot]);
+            if (lane == 0) mbar_arrive(&bar[C::B_W_FULL + slot]);
         }
-        if (lane == 0 && slice == 0) {
+        if (warp == 2 && lane == 0 && slice == 0) {
             double *sc = p.segS + ((size_t)g * p.BH + bh) * 2;
             sc[0] = Fseg;
             sc[1] = Fseg + ustar;
         }
-    } else if (warp == 3) {
-        // ===================== n_seg = sum_t w_t k_t =====================
-        constexpr int NPL = DQK / 32;   // columns per lane
-        const int j0 = lane * NPL;
-        const uint32_t box = j0 >> 6, chk = (j0 & 63) >> 3, within = (j0 & 7) * 2;
-        float nacc[NPL];
-#pragma unroll
-        for (int i = 0; i < NPL; ++i) nacc[i] = 0.f;
-        bool alive = true;
-        for (int c = 0; c < NC; ++c) {
-            const int s = c % kStages, slot = c % kRing;
-            alive = waitw(sh, &bar[S_KV_FULL + s], (c / kStages) & 1, kWhereSumKv) &&
-                    waitw(sh, &bar[S_W_FULL + slot], (c / kRing) & 1, kWhereSumW);
-            if (!alive) break;
-            const uint8_t *Ks = sm + C::OFF_K + s * C::K_BYTES + box * 8192 + within;
-            const float *w = wring + slot * kL;
-#pragma unroll 4
-            for (int t = 0; t < kL; ++t) {
-                const uint8_t *src = Ks + sw128_offset(t, chk);
-                const float wt = w[t];
-                if (NPL == 8) {
-                    float x[8];
-                    unpack_bf16x8(*reinterpret_cast<const uint4 *>(src), x);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) nacc[i % NPL] = fmaf(wt, x[i], nacc[i % NPL]);
-                } else if (NPL == 4) {
-                    const uint2 u = *reinterpret_cast<const uint2 *>(src);
-                    const float x[4] = {bf_lo(u.x), bf_hi(u.x), bf_lo(u.y), bf_hi(u.y)};
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) nacc[i % NPL] = fmaf(wt, x[i], nacc[i % NPL]);
-                } else {
-                    const uint32_t u = *reinterpret_cast<const uint32_t *>(src);
-                    const float x[2] = {bf_lo(u), bf_hi(u)};
-#pragma unroll
-                    for (int i = 0; i < 2; ++i) nacc[i % NPL] = fmaf(wt, x[i], nacc[i % NPL]);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) {
-                mbar_arrive(&bar[S_KV_EMPTY + s]);
-                mbar_arrive(&bar[S_W_EMPTY + slot]);
-            }
-        }
-        if (alive && slice == 0) {
-            float *dst = p.segN + ((size_t)g * p.BH + bh) * DQK + j0;
-#pragma unroll
-            for (int i = 0; i < NPL; ++i) dst[i] = nacc[i];
-        }
     } else {
-        // ===================== w V in place; read-out of C_seg =====================
+        // ===================== w V in place, n_seg; read-out of C_seg =====================
+        // Thread t128 also owns columns t128 (+ 128) of n_seg (the first value slice only).
+        constexpr int NJ = (DQK + 127) / 128;
         const int t128 = tid - 128;
+        float nacc[NJ];
+#pragma unroll
+        for (int i = 0; i < NJ; ++i) nacc[i] = 0.f;
         bool alive = true;
         for (int c = 0; c < NC; ++c) {
-            const int s = c % kStages, slot = c % kRing;
-            alive = alive && waitw(sh, &bar[S_KV_FULL + s], (c / kStages) & 1, kWhereSumKv) &&
-                    waitw(sh, &bar[S_W_FULL + slot], (c / kRing) & 1, kWhereSumW);
+            const int s = c % C::STAGES, slot = c % kRing;
+            alive = alive && waitw(sh, &bar[C::B_KV_FULL + s], (c / C::STAGES) & 1, kWhereSumKv) &&
+                    waitw(sh, &bar[C::B_W_FULL + slot], (c / kRing) & 1, kWhereSumW);
+            const float *w = wring + slot * kL;
             if (alive) {
-                scale_v_rows(sm + C::OFF_V + s * C::V_BYTES, wring + slot * kL, t128);
+                scale_v_rows(sm + C::OFF_V + s * C::V_BYTES, w, t128);
                 fence_proxy_async_smem();   // the MMA (async proxy) reads what these stores wrote
             }
             // unconditional: every warp of the group takes every barrier, even after
             // another warp of it gave up
             named_barrier(1, 128);
+            if (t128 == 0 && alive) mbar_arrive(&bar[C::B_VS + s]);
+            if (alive && slice == 0) {
+                const uint8_t *Ks = sm + C::OFF_K + s * C::K_BYTES;
+#pragma unroll
+                for (int i = 0; i < NJ; ++i) {
+                    const int j = t128 + 128 * i;
+                    if (j < DQK) {
+                        const uint8_t *col = Ks + (j >> 6) * 8192 + (j & 7) * 2;
+                        const uint32_t chk = (j & 63) >> 3;
+                        float acc = nacc[i];
+#pragma unroll 8
+                        for (int t = 0; t < kL; ++t)
+                            acc = fmaf(w[t], __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
+                                                 col + sw128_offset(t, chk))),
+                                       acc);
+                        nacc[i] = acc;
+                    }
+                }
+            }
+            named_barrier(1, 128);
             if (t128 == 0 && alive) {
-                mbar_arrive(&bar[S_VS + s]);
-                mbar_arrive(&bar[S_W_EMPTY + slot]);
+                mbar_arrive(&bar[C::B_W_EMPTY + slot]);
+                mbar_arrive(&bar[C::B_KV_EMPTY + s]);
             }
         }
-        alive = alive && waitw(sh, &bar[S_DONE], 0, kWhereSumDone);
+        if (alive && slice == 0) {
+#pragma unroll
+            for (int i = 0; i < NJ; ++i) {
+                const int j = t128 + 128 * i;
+                if (j < DQK) p.segN[((size_t)g * p.BH + bh) * DQK + j] = nacc[i];
+            }
+        }
+        alive = alive && waitw(sh, &bar[C::B_DONE], 0, kWhereSumDone);
         const int v = v0 + t128;
         if (alive && v < p.dv) {   // warp-uniform: d_v is a multiple of 64
             tc_fence_after();
@@ -335,8 +353,11 @@ struct CombineParams {
 
 // Entry states, in place over the summaries: slot g becomes the state entering
 // segment g+1.  One thread per 4 consecutive floats of (C, n) of one sequence;
-// every thread runs the scalar chain of gauges itself, in float64.
+// every thread runs the scalar chain of gauges itself, in float64.  The loads of
+// a batch of segments are issued before any of them is combined, so that the
+// chain waits on one memory round trip per batch, not per segment.
 __global__ void __launch_bounds__(kCombineThreads) seg_combine_kernel(const CombineParams p) {
+    constexpr int kBatch = 8;
     const int bh = blockIdx.y;
     const int nC4 = p.dv * p.dqk / 4, n4 = nC4 + p.dqk / 4;
     const int e4 = blockIdx.x * kCombineThreads + threadIdx.x;
@@ -346,19 +367,36 @@ __global__ void __launch_bounds__(kCombineThreads) seg_combine_kernel(const Comb
     if (isC && p.C0) x = reinterpret_cast<const float4 *>(p.C0 + (size_t)bh * p.dv * p.dqk)[e4];
     if (!isC && p.n0) x = reinterpret_cast<const float4 *>(p.n0 + (size_t)bh * p.dqk)[e4 - nC4];
     double m = p.m0 ? (double)p.m0[bh] : 0.0;
-    for (int g = 0; g < p.nsum; ++g) {
-        const double F = p.segS[((size_t)g * p.BH + bh) * 2], ms = p.segS[((size_t)g * p.BH + bh) * 2 + 1];
-        // the new gauge, rounded to the fp32 m the chunkwise kernel reads, so that the
-        // state handed on is exactly in the gauge it is labelled with
-        const double mp = (double)(float)fmax(F + m, ms);
-        const float a = (float)exp(F + m - mp), b = (float)exp(ms - mp);
-        float4 *slot = isC ? reinterpret_cast<float4 *>(p.segC + ((size_t)g * p.BH + bh) * p.dv * p.dqk) + e4
-                           : reinterpret_cast<float4 *>(p.segN + ((size_t)g * p.BH + bh) * p.dqk) + (e4 - nC4);
-        const float4 y = *slot;
-        x = make_float4(fmaf(a, x.x, b * y.x), fmaf(a, x.y, b * y.y), fmaf(a, x.z, b * y.z), fmaf(a, x.w, b * y.w));
-        *slot = x;
-        if (e4 == 0) p.segM[(size_t)g * p.BH + bh] = (float)mp;
-        m = mp;
+    auto slot = [&](int g) {
+        return isC ? reinterpret_cast<float4 *>(p.segC + ((size_t)g * p.BH + bh) * p.dv * p.dqk) + e4
+                   : reinterpret_cast<float4 *>(p.segN + ((size_t)g * p.BH + bh) * p.dqk) + (e4 - nC4);
+    };
+    for (int g0 = 0; g0 < p.nsum; g0 += kBatch) {
+        float4 y[kBatch];
+        double F[kBatch], ms[kBatch];
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            if (g0 + j < p.nsum) {
+                const size_t k = ((size_t)(g0 + j) * p.BH + bh) * 2;
+                y[j] = *slot(g0 + j);
+                F[j] = p.segS[k];
+                ms[j] = p.segS[k + 1];
+            }
+        }
+#pragma unroll
+        for (int j = 0; j < kBatch; ++j) {
+            if (g0 + j < p.nsum) {
+                // the new gauge, rounded to the fp32 m the chunkwise kernel reads, so that
+                // the state handed on is exactly in the gauge it is labelled with
+                const double mp = (double)(float)fmax(F[j] + m, ms[j]);
+                const float a = (float)exp(F[j] + m - mp), b = (float)exp(ms[j] - mp);
+                x = make_float4(fmaf(a, x.x, b * y[j].x), fmaf(a, x.y, b * y[j].y), fmaf(a, x.z, b * y[j].z),
+                                fmaf(a, x.w, b * y[j].w));
+                *slot(g0 + j) = x;
+                if (e4 == 0) p.segM[(size_t)(g0 + j) * p.BH + bh] = (float)mp;
+                m = mp;
+            }
+        }
     }
 }
 
@@ -418,6 +456,7 @@ SegPlan segment_plan(const FwdArgs &a) {
     const long long fit = sm_count() / blocks;   // segments per sequence that still fit one wave
     int G = (int)std::min<long long>(fit, NC / kMinSegChunks);
     if (G < 2) return sp;
+    G = std::max(G, (NC + kMaxSegChunks - 1) / kMaxSegChunks);   // no segment longer than kMaxSegChunks
     sp.seg_chunks = (NC + G - 1) / G;
     G = (NC + sp.seg_chunks - 1) / sp.seg_chunks;
     if (G < 2) return sp;
