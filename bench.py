@@ -53,12 +53,14 @@ def peaks():
     return 6650.0, 1590.0, 1400.0, "fallback"
 
 
-def algorithmic(w, L=64):
+def algorithmic(w, L=64, gated=False):
     """Bytes and flops of one step (counting convention of the design notes).
 
     Sequence workloads: one forward over B*H*T head-tokens; inputs, h~ and the
     final state (plus the initial state when one is read).  Decode: one step
     over B*H heads; the state is read and written once, plus the step's vectors.
+    gated: the fused output stage, bf16 o~ read and bf16 h written instead of
+    fp32 h~.
     """
     e = 2 if w.dtype == "bf16" else 4
     state = w.d_qk * w.d_v + w.d_qk + 1
@@ -68,7 +70,8 @@ def algorithmic(w, L=64):
         flops = BH * (5 * w.d_qk * w.d_v + 4 * w.d_qk)
         return bytes_, flops
     N = w.B * w.H * w.T
-    bytes_ = N * ((2 * w.d_qk + w.d_v) * e + 8 + 4 * w.d_v) + w.B * w.H * state * 4
+    out_bytes = (2 + 2) * w.d_v if gated else 4 * w.d_v
+    bytes_ = N * ((2 * w.d_qk + w.d_v) * e + 8 + out_bytes) + w.B * w.H * state * 4
     if w.state != "zero":
         bytes_ += w.B * w.H * state * 4
     flops = N * (4 * w.d_qk * w.d_v + L * (w.d_qk + w.d_v))
@@ -179,9 +182,10 @@ def config_of(w, extra=None):
     return c
 
 
-def cpu_baseline(w, inp, budget_s=12.0):
+def cpu_baseline(w, inp, budget_s=12.0, gated=False):
     """Time the float64 oracle on a bounded sample of the workload, all host
-    threads.  Returns the rate in the workload's tokens/s."""
+    threads.  Returns the rate in the workload's tokens/s.  gated: the oracle's
+    output gate follows the recurrence on the sample."""
     import oracle
     threads = oracle.default_threads()
     flat = lambda x: None if x is None else x.reshape((w.B * w.H,) + x.shape[2:])
@@ -215,9 +219,15 @@ def cpu_baseline(w, inp, budget_s=12.0):
     per_head_token = (time.perf_counter() - t0) / Tp
     nheads = int(max(1, min(w.B * w.H, threads * budget_s / max(per_head_token * w.T, 1e-9))))
     hs = list(range(nheads))
+    o_s = None
+    if gated:
+        from xlstm_mlstm_matrix_b200 import inputs as _inputs
+        o_s = sel(_inputs.output_gate_pre(w, "bf16"), hs)
     t0 = time.perf_counter()
-    oracle.forward(*(sel(inp[n], hs) for n in ("q", "k", "v", "i_pre", "f_pre", "C0", "n0", "m0")),
-                   qk_scale=inp["qk_scale"], threads=threads)
+    h = oracle.forward(*(sel(inp[n], hs) for n in ("q", "k", "v", "i_pre", "f_pre", "C0", "n0", "m0")),
+                       qk_scale=inp["qk_scale"], threads=threads)[0]
+    if gated:
+        oracle.output_gate(h, o_s)
     dt = time.perf_counter() - t0
     tokens = nheads * w.T / w.H          # head-tokens / heads per token
     return {"value": tokens / dt, "unit": UNIT, "cores": min(threads, nheads), "kind": "oracle",
@@ -273,24 +283,27 @@ def run_reference(args, rank, world):
     budget = max(0.5, min(args.ref_budget, 120.0 / max(1, args.steps)))
     vals = []
     cb = None
+    gated = args.output == "gated-bf16" and not w.steps
     for _ in range(max(1, args.steps)):
-        cb = cpu_baseline(w, inp, budget_s=budget)
+        cb = cpu_baseline(w, inp, budget_s=budget, gated=gated)
         vals.append(cb["value"])
     value = statistics.median(vals)
     cb["value"] = value
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": 1e3 * tokens_per_step(w) / value,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-            "data": "synthetic", "impl": "reference", "config": config_of(w),
+            "data": "synthetic", "impl": "reference",
+            "config": config_of(w, {"output": "gated-bf16"} if gated else None),
             "cpu_baseline": cb,
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
 class _Sequence:
-    """One chunkwise forward over the whole batch per step."""
+    """One chunkwise forward over the whole batch per step (gated: through the
+    fused output stage, bf16 o~ in and bf16 h out)."""
 
-    def __init__(self, w, inp, dev, stream):
+    def __init__(self, w, inp, dev, stream, gated=False):
         import torch
         from xlstm_mlstm_matrix_b200 import capi
         self.w, self.inp = w, inp
@@ -299,7 +312,12 @@ class _Sequence:
             torch.from_numpy(x).to(dev).to(torch.bfloat16) if b else torch.from_numpy(x).to(dev))
         self.ins = [dev_t(inp[n], bf) for n in ("q", "k", "v")] + \
                    [dev_t(inp[n], False) for n in ("i_pre", "f_pre", "C0", "n0", "m0")]
-        self.outs = [torch.empty(w.B, w.H, w.T, w.d_v, device=dev),
+        self.gated = gated
+        if gated:
+            from xlstm_mlstm_matrix_b200 import inputs as _inputs
+            self.ins.append(dev_t(_inputs.output_gate_pre(w, "bf16"), True))
+        self.outs = [torch.empty(w.B, w.H, w.T, w.d_v, device=dev,
+                                 dtype=torch.bfloat16 if gated else torch.float32),
                      torch.empty(w.B, w.H, w.d_v, w.d_qk, device=dev),
                      torch.empty(w.B, w.H, w.d_qk, device=dev), torch.empty(w.B, w.H, device=dev)]
         self.desc = capi.make_desc(w.B, w.H, w.T, w.d_qk, w.d_v,
@@ -309,15 +327,21 @@ class _Sequence:
         wsb = capi.xlstm_mlstm_workspace_size_parallel(self.desc)
         segmented = wsb > capi.xlstm_mlstm_workspace_size(self.desc)
         self.ws = torch.zeros(wsb, device=dev, dtype=torch.uint8)
-        self.fn = capi.load().xlstm_mlstm_fwd_chunkwise
         import ctypes
         P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
-        self.argv = (ctypes.byref(self.desc), *(P(t) for t in self.ins), *(P(t) for t in self.outs),
-                     P(self.ws), wsb, ctypes.c_void_p(stream.cuda_stream))
+        if gated:
+            self.fn = capi.load().xlstm_mlstm_fwd_chunkwise_out
+            self.ostage = capi.xlstm_mlstm_output_t(self.ins[-1].data_ptr(), capi.XLSTM_BF16, capi.XLSTM_BF16)
+            self.argv = (ctypes.byref(self.desc), ctypes.byref(self.ostage), *(P(t) for t in self.ins[:-1]),
+                         *(P(t) for t in self.outs), P(self.ws), wsb, ctypes.c_void_p(stream.cuda_stream))
+        else:
+            self.fn = capi.load().xlstm_mlstm_fwd_chunkwise
+            self.argv = (ctypes.byref(self.desc), *(P(t) for t in self.ins), *(P(t) for t in self.outs),
+                         P(self.ws), wsb, ctypes.c_void_p(stream.cuda_stream))
         self.stream = stream
         self.kernel = "chunkwise (segment summaries + combine + chunkwise)" if segmented else "chunkwise"
         self.launches = 3 if segmented else 1   # kernels per call
-        self.name = "xlstm_mlstm_fwd_chunkwise"
+        self.name = "xlstm_mlstm_fwd_chunkwise_out" if gated else "xlstm_mlstm_fwd_chunkwise"
 
     def step(self, i):
         st = self.fn(*self.argv)
@@ -409,7 +433,10 @@ def run_ours(args, rank, world, local_rank):
     w = workload_for_rank(args.workload, rank, args.B, args.H, args.T)
     inp = make_inputs(w)
     stream = torch.cuda.Stream(dev)
-    job = _Decode(w, inp, dev, stream) if w.steps else _Sequence(w, inp, dev, stream)
+    gated = args.output == "gated-bf16"
+    if gated and w.steps:
+        raise SystemExit("--output gated-bf16 applies to the sequence workloads")
+    job = _Decode(w, inp, dev, stream) if w.steps else _Sequence(w, inp, dev, stream, gated=gated)
 
     dist = None
     if world > 1:
@@ -446,7 +473,7 @@ def run_ours(args, rank, world, local_rank):
 
     tokens = tokens_per_step(w)
     value = job_rate(tokens, world, ms)
-    bytes_, flops = algorithmic(w)
+    bytes_, flops = algorithmic(w, gated=gated)
     hbm, bf16_peak, _, peak_src = peaks()
     achieved_gbs = bytes_ / (ms * 1e-3) / 1e9
     src_sha = kernel_source_sha()
@@ -489,10 +516,13 @@ def run_ours(args, rank, world, local_rank):
     if rank == 0:
         l2 = (f"inputs larger than L2 ({bytes_ / 1e9:.2f} GB per step vs 126 MB L2)"
               if bytes_ > 4 * 126e6 else "working set near L2 size; no flush")
-        extra = {"inputs": "bf16 q/k/v, fp32 gates; fp32 h and state", "l2": l2,
+        extra = {"inputs": ("bf16 q/k/v and o~, fp32 gates; bf16 h = sigmoid(o~) h~ (output stage fused), fp32 state"
+                            if gated else "bf16 q/k/v, fp32 gates; fp32 h and state"), "l2": l2,
                  "parallelism": f"replicas x{world} (independent heads)"}
         if not w.steps:
             extra["chunk"] = 64
+        if gated:
+            extra["output"] = "gated-bf16"
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
@@ -511,7 +541,7 @@ def run_ours(args, rank, world, local_rank):
             "kernel_source_sha": src_sha,
         }
         if world == 1 and not args.no_cpu_baseline:
-            line["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.ref_budget)
+            line["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.ref_budget, gated=gated)
         print(json.dumps(line), flush=True)
 
 
@@ -526,6 +556,8 @@ def main():
                     default=DEFAULT_WORKLOAD)
     ap.add_argument("--ref-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--output", choices=["plain", "gated-bf16"], default="plain",
+                    help="gated-bf16: the fused output stage (h = sigmoid(o~) h~, bf16 o~ and h)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
     ap.add_argument("--H", type=int, default=0, help="override the head count (profiling)")

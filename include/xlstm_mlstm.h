@@ -114,6 +114,39 @@ XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise(
     void *workspace, size_t workspace_bytes, cudaStream_t stream);
 
 /*
+ * Output stage of xlstm_mlstm_fwd_chunkwise_out (xLSTM page, "mLSTM (matrix
+ * LSTM)" eq. 3, h_t = o_t * h~_t, with o_t = sigmoid(o~_t) as in the o_t line of
+ * the page's forward_recurrent listing, the projection removed).
+ *   o_pre   : [B][H][T][d_v] output-gate pre-activations o~ (device), or NULL
+ *             for no gate (h = h~).  An input: must not overlap any output.
+ *   o_dtype : XLSTM_F32 or XLSTM_BF16, the element type of o_pre.
+ *   h_dtype : XLSTM_F32 or XLSTM_BF16, the element type of h_out (bf16: rounded
+ *             to nearest even from the fp32 result).
+ */
+typedef struct {
+    const void *o_pre;
+    xlstm_dtype_t o_dtype;
+    xlstm_dtype_t h_dtype;
+} xlstm_mlstm_output_t;
+
+/*
+ * xlstm_mlstm_fwd_chunkwise with the output stage fused into the epilogue:
+ * h_out[b][h][t][:] = sigmoid(o_pre[b][h][t][:]) * h~_t (elementwise), stored as
+ * out->h_dtype.  out == NULL is xlstm_mlstm_fwd_chunkwise exactly.  Same
+ * arguments, rules, workspace and status block otherwise; h_out holds
+ * B*H*T*d_v elements of h_dtype.  Invalid dtypes or a misaligned o_pre give
+ * XLSTM_ERR_INVALID_ARG.  The state outputs are the recurrence's, untouched by
+ * the gate.
+ */
+XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise_out(
+    const xlstm_mlstm_desc_t *desc, const xlstm_mlstm_output_t *out,
+    const void *q, const void *k, const void *v,
+    const float *i_pre, const float *f_pre,
+    const float *C_in, const float *n_in, const float *m_in,
+    void *h_out, float *C_out, float *n_out, float *m_out,
+    void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Recurrent forward over a whole sequence: the recurrence above evaluated one
  * token at a time with the state held on chip (O(1) state memory per head,
  * O(T) time).  Same arguments and rules as xlstm_mlstm_fwd_chunkwise;

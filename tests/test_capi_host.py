@@ -124,6 +124,32 @@ def test_workspace_and_chunk_rules(lib):
     assert call(d) == capi.XLSTM_ERR_UNSUPPORTED
 
 
+def test_output_stage_arguments_checked(lib):
+    """xlstm_mlstm_fwd_chunkwise_out: bad dtypes, a misaligned o_pre and an o_pre
+    that overlaps h are refused before any device work; NULL out is the plain call."""
+    d = capi.make_desc(2, 2, 64, 64, 64, capi.XLSTM_BF16, 1.0, 64)
+    a = dict(FAKE)
+    h_bytes16 = 2 * 2 * 64 * 64 * 2
+
+    def call_out(o, odt, hdt, h=a["h"]):
+        out = capi.xlstm_mlstm_output_t(o, odt, hdt)
+        return capi.xlstm_mlstm_fwd_chunkwise_out(d, out, a["q"], a["k"], a["v"], a["i"], a["f"], None, None, None,
+                                                  h, None, None, None, a["ws"], 256)
+    assert call_out(0x70000, capi.XLSTM_BF16, 7) == capi.XLSTM_ERR_INVALID_ARG
+    assert call_out(0x70000, 9, capi.XLSTM_F32) == capi.XLSTM_ERR_INVALID_ARG
+    assert call_out(0x70002, capi.XLSTM_BF16, capi.XLSTM_F32) == capi.XLSTM_ERR_INVALID_ARG
+    # o_pre inside h (bf16 h: h_bytes16 bytes from 0x60000)
+    assert call_out(0x60000 + h_bytes16 - 16, capi.XLSTM_BF16, capi.XLSTM_BF16) == capi.XLSTM_ERR_INVALID_ARG
+    # the same o_pre just past a bf16 h is fine as far as overlap goes; it fails later only on the
+    # (fake) workspace, which the argument checks do not reach: use a too-small workspace instead
+    out = capi.xlstm_mlstm_output_t(0x60000 + h_bytes16, capi.XLSTM_BF16, capi.XLSTM_BF16)
+    assert capi.xlstm_mlstm_fwd_chunkwise_out(d, out, a["q"], a["k"], a["v"], a["i"], a["f"], None, None, None,
+                                              a["h"], None, None, None, a["ws"], 16) == capi.XLSTM_ERR_WORKSPACE
+    # NULL out: the plain call's checks
+    assert capi.xlstm_mlstm_fwd_chunkwise_out(d, None, a["q"], a["k"], a["v"], a["i"], a["f"], None, None, None,
+                                              None, None, None, None, a["ws"], 256) == capi.XLSTM_ERR_INVALID_ARG
+
+
 def test_step_rejects_partial_in_place(lib):
     d = capi.make_desc(2, 2, 1, 32, 32)
     C, n, m = 0x70000, 0x80000, 0x90000

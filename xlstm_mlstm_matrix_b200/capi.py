@@ -21,13 +21,18 @@ XLSTM_F32, XLSTM_BF16 = 0, 1
 EXPORTED = ("xlstm_mlstm_fwd_chunkwise", "xlstm_mlstm_fwd_recurrent", "xlstm_mlstm_step",
             "xlstm_mlstm_workspace_size", "xlstm_mlstm_workspace_status", "xlstm_status_string",
             "xlstm_mlstm_version", "xlstm_mlstm_chunkwise_kernel", "xlstm_mlstm_test_timeout_next",
-            "xlstm_mlstm_fwd_chunkwise_noalloc", "xlstm_mlstm_workspace_size_parallel")
+            "xlstm_mlstm_fwd_chunkwise_noalloc", "xlstm_mlstm_workspace_size_parallel",
+            "xlstm_mlstm_fwd_chunkwise_out")
 
 
 class xlstm_mlstm_desc_t(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int32), ("H", ctypes.c_int32), ("T", ctypes.c_int32),
                 ("d_qk", ctypes.c_int32), ("d_v", ctypes.c_int32), ("qkv_dtype", ctypes.c_int32),
                 ("qk_scale", ctypes.c_float), ("chunk", ctypes.c_int32)]
+
+
+class xlstm_mlstm_output_t(ctypes.Structure):
+    _fields_ = [("o_pre", ctypes.c_void_p), ("o_dtype", ctypes.c_int32), ("h_dtype", ctypes.c_int32)]
 
 
 class XlstmError(RuntimeError):
@@ -53,6 +58,8 @@ def load(path: str = LIB_PATH):
     for name in ("xlstm_mlstm_fwd_chunkwise", "xlstm_mlstm_fwd_recurrent"):
         getattr(lib, name).argtypes = seq
         getattr(lib, name).restype = st
+    lib.xlstm_mlstm_fwd_chunkwise_out.argtypes = [dp, ctypes.POINTER(xlstm_mlstm_output_t)] + [vp] * 12 + [vp, sz, vp]
+    lib.xlstm_mlstm_fwd_chunkwise_out.restype = st
     lib.xlstm_mlstm_fwd_chunkwise_noalloc.argtypes = [dp] + [vp] * 12 + [vp]
     lib.xlstm_mlstm_fwd_chunkwise_noalloc.restype = st
     lib.xlstm_mlstm_step.argtypes = [dp] + [vp] * 12 + [vp]
@@ -124,6 +131,15 @@ def xlstm_mlstm_fwd_recurrent(desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in, h_o
         _s(stream))
 
 
+def xlstm_mlstm_fwd_chunkwise_out(desc, out, q, k, v, i_pre, f_pre, C_in, n_in, m_in, h_out, C_out,
+                                  n_out, m_out, workspace, workspace_bytes, stream=None) -> int:
+    """out: an xlstm_mlstm_output_t or None."""
+    return load().xlstm_mlstm_fwd_chunkwise_out(
+        ctypes.byref(desc), None if out is None else ctypes.byref(out), _p(q), _p(k), _p(v), _p(i_pre),
+        _p(f_pre), _p(C_in), _p(n_in), _p(m_in), _p(h_out), _p(C_out), _p(n_out), _p(m_out), _p(workspace),
+        int(workspace_bytes), _s(stream))
+
+
 def xlstm_mlstm_step(desc, q, k, v, i_pre, f_pre, C, n, m, h_out, C_new, n_new, m_new,
                      stream=None) -> int:
     return load().xlstm_mlstm_step(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(i_pre), _p(f_pre),
@@ -184,20 +200,27 @@ def _dtype_code(t):
 
 
 def fwd(q, k, v, i_pre, f_pre, state=None, qk_scale=None, chunk=0, kind="chunkwise",
-        stream=None, workspace=None, out=None, parallel=True):
+        stream=None, workspace=None, out=None, parallel=True, o_pre=None, h_dtype=None):
     """Sequence forward through the C ABI.  q, k [B,H,T,dqk], v [B,H,T,dv]
     (bf16 or fp32, CUDA, contiguous), i_pre/f_pre [B,H,T] fp32; state is None
     or (C [B,H,dv,dqk], n [B,H,dqk], m [B,H]).  Returns (h, (C, n, m)).
     Without a given workspace, the chunkwise call gets one large enough for the
-    segment-parallel evaluation of long sequences (parallel=False: the minimum)."""
+    segment-parallel evaluation of long sequences (parallel=False: the minimum).
+    o_pre [B,H,T,dv] (bf16 or fp32) applies the output gate, h = sigmoid(o_pre) h~,
+    and h_dtype (torch.bfloat16 or torch.float32) picks h's type: both through
+    xlstm_mlstm_fwd_chunkwise_out (chunkwise only)."""
     import torch
     B, H, T, dqk = q.shape
     dv = v.shape[-1]
     scale = (dqk ** -0.5) if qk_scale is None else float(qk_scale)
     desc = make_desc(B, H, T, dqk, dv, _dtype_code(q), scale, chunk)
     dev = q.device
+    staged = o_pre is not None or h_dtype is not None
+    if staged and kind != "chunkwise":
+        raise ValueError("the output stage is fused into the chunkwise call only")
+    hdt = torch.float32 if h_dtype is None else h_dtype
     if out is None:
-        h = torch.empty(B, H, T, dv, device=dev, dtype=torch.float32)
+        h = torch.empty(B, H, T, dv, device=dev, dtype=hdt)
         C1 = torch.empty(B, H, dv, dqk, device=dev, dtype=torch.float32)
         n1 = torch.empty(B, H, dqk, device=dev, dtype=torch.float32)
         m1 = torch.empty(B, H, device=dev, dtype=torch.float32)
@@ -209,8 +232,15 @@ def fwd(q, k, v, i_pre, f_pre, state=None, qk_scale=None, chunk=0, kind="chunkwi
         if workspace is None:
             need = (xlstm_mlstm_workspace_size_parallel if parallel else xlstm_mlstm_workspace_size)(desc)
             workspace = torch.empty(max(256, need), device=dev, dtype=torch.uint8)
-        st = xlstm_mlstm_fwd_chunkwise(desc, q, k, v, i_pre, f_pre, C0, n0, m0, h, C1, n1, m1,
-                                       workspace, workspace.numel(), stream)
+        if staged:
+            ostage = xlstm_mlstm_output_t(None if o_pre is None else o_pre.data_ptr(),
+                                          XLSTM_F32 if o_pre is None else _dtype_code(o_pre),
+                                          XLSTM_BF16 if hdt == torch.bfloat16 else XLSTM_F32)
+            st = xlstm_mlstm_fwd_chunkwise_out(desc, ostage, q, k, v, i_pre, f_pre, C0, n0, m0, h, C1, n1,
+                                               m1, workspace, workspace.numel(), stream)
+        else:
+            st = xlstm_mlstm_fwd_chunkwise(desc, q, k, v, i_pre, f_pre, C0, n0, m0, h, C1, n1, m1,
+                                           workspace, workspace.numel(), stream)
     elif kind == "recurrent":
         st = xlstm_mlstm_fwd_recurrent(desc, q, k, v, i_pre, f_pre, C0, n0, m0, h, C1, n1, m1,
                                        None, 0, stream)

@@ -37,23 +37,27 @@ bool dims_ok(const xlstm_mlstm_desc_t *d) {
 size_t elem(const xlstm_mlstm_desc_t *d) { return d->qkv_dtype == XLSTM_BF16 ? 2 : 4; }
 
 // Shared validation of the two sequence calls.
+// h_elem: bytes per element of h; o (optional input, o_elem bytes per element) is
+// the output-gate pre-activation tensor of the chunkwise output stage.
 xlstm_status_t check_sequence(const xlstm_mlstm_desc_t *d, const void *q, const void *k,
                               const void *v, const float *ig, const float *fg, const float *C0,
-                              const float *n0, const float *m0, const float *h, const float *C1,
-                              const float *n1, const float *m1) {
+                              const float *n0, const float *m0, const void *h, const float *C1,
+                              const float *n1, const float *m1, size_t h_elem = 4,
+                              const void *o = nullptr, size_t o_elem = 0) {
     if (!d || !dims_ok(d)) return XLSTM_ERR_INVALID_ARG;
     const int ns = (C0 != nullptr) + (n0 != nullptr) + (m0 != nullptr);
     if (ns != 0 && ns != 3) return XLSTM_ERR_INVALID_ARG;
     if (d->T > 0 && (!q || !k || !v || !ig || !fg || !h)) return XLSTM_ERR_INVALID_ARG;
-    const void *all[] = {q, k, v, ig, fg, C0, n0, m0, h, C1, n1, m1};
+    const void *all[] = {q, k, v, ig, fg, C0, n0, m0, h, C1, n1, m1, o};
     for (const void *p : all)
         if (!aligned16(p)) return XLSTM_ERR_INVALID_ARG;
     const size_t BH = (size_t)d->B * d->H, T = (size_t)d->T;
     const size_t e = elem(d);
     const Range ins[] = {rg(q, BH * T * d->d_qk * e), rg(k, BH * T * d->d_qk * e),
                          rg(v, BH * T * d->d_v * e), rg(ig, BH * T * 4), rg(fg, BH * T * 4),
-                         rg(C0, BH * d->d_v * d->d_qk * 4), rg(n0, BH * d->d_qk * 4), rg(m0, BH * 4)};
-    const Range outs[] = {rg(h, BH * T * d->d_v * 4), rg(C1, BH * d->d_v * d->d_qk * 4),
+                         rg(C0, BH * d->d_v * d->d_qk * 4), rg(n0, BH * d->d_qk * 4), rg(m0, BH * 4),
+                         rg(o, BH * T * d->d_v * o_elem)};
+    const Range outs[] = {rg(h, BH * T * d->d_v * h_elem), rg(C1, BH * d->d_v * d->d_qk * 4),
                           rg(n1, BH * d->d_qk * 4), rg(m1, BH * 4)};
     for (const Range &o : outs) {
         for (const Range &i : ins)
@@ -105,20 +109,18 @@ size_t xlstm_mlstm_workspace_size_parallel(const xlstm_mlstm_desc_t *desc) {
     return kWorkspaceBytes + (sp.nseg > 1 ? sp.bytes : 0);
 }
 
-xlstm_status_t xlstm_mlstm_fwd_chunkwise(const xlstm_mlstm_desc_t *desc, const void *q,
-                                         const void *k, const void *v, const float *i_pre,
-                                         const float *f_pre, const float *C_in, const float *n_in,
-                                         const float *m_in, float *h_out, float *C_out,
-                                         float *n_out, float *m_out, void *workspace,
-                                         size_t workspace_bytes, cudaStream_t stream) {
-    xlstm_status_t st = check_sequence(desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in, h_out,
-                                       C_out, n_out, m_out);
+}  // extern "C"
+
+namespace {
+
+// The chunkwise call behind both entry points; a is packed, st the argument check.
+xlstm_status_t run_chunkwise(const xlstm_mlstm_desc_t *desc, FwdArgs a, xlstm_status_t st, void *workspace,
+                             size_t workspace_bytes, cudaStream_t stream) {
     if (st != XLSTM_OK) return st;
     const int L = desc->chunk ? desc->chunk : 64;
     if (L != 16 && L != 32 && L != 64) return XLSTM_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < xlstm_mlstm_workspace_size(desc)) return XLSTM_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return XLSTM_ERR_INVALID_ARG;
-    FwdArgs a = pack(desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in, h_out, C_out, n_out, m_out);
     a.status = static_cast<int32_t *>(workspace);
     if (cudaMemsetAsync(workspace, 0, 16, stream) != cudaSuccess) return XLSTM_ERR_CUDA;
     if (a.T == 0) return pass_state_through(a, stream);
@@ -131,6 +133,47 @@ xlstm_status_t xlstm_mlstm_fwd_chunkwise(const xlstm_mlstm_desc_t *desc, const v
     cudaError_t e = xlstm::chunkwise_tc_supported(a) ? xlstm::launch_chunkwise_tc(a, stream)
                                                      : xlstm::launch_chunkwise_simt(a, stream);
     return e == cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+xlstm_status_t xlstm_mlstm_fwd_chunkwise(const xlstm_mlstm_desc_t *desc, const void *q,
+                                         const void *k, const void *v, const float *i_pre,
+                                         const float *f_pre, const float *C_in, const float *n_in,
+                                         const float *m_in, float *h_out, float *C_out,
+                                         float *n_out, float *m_out, void *workspace,
+                                         size_t workspace_bytes, cudaStream_t stream) {
+    const xlstm_status_t st = check_sequence(desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in, h_out,
+                                             C_out, n_out, m_out);
+    if (st != XLSTM_OK) return st;
+    return run_chunkwise(desc, pack(desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in, h_out, C_out, n_out, m_out), st,
+                         workspace, workspace_bytes, stream);
+}
+
+xlstm_status_t xlstm_mlstm_fwd_chunkwise_out(const xlstm_mlstm_desc_t *desc, const xlstm_mlstm_output_t *out,
+                                             const void *q, const void *k, const void *v, const float *i_pre,
+                                             const float *f_pre, const float *C_in, const float *n_in,
+                                             const float *m_in, void *h_out, float *C_out, float *n_out,
+                                             float *m_out, void *workspace, size_t workspace_bytes,
+                                             cudaStream_t stream) {
+    xlstm::OutStage os;
+    if (out) {
+        const bool ok_o = out->o_pre == nullptr || out->o_dtype == XLSTM_F32 || out->o_dtype == XLSTM_BF16;
+        if (!ok_o || (out->h_dtype != XLSTM_F32 && out->h_dtype != XLSTM_BF16)) return XLSTM_ERR_INVALID_ARG;
+        os.o = out->o_pre;
+        os.o_bf16 = out->o_pre && out->o_dtype == XLSTM_BF16;
+        os.h_bf16 = out->h_dtype == XLSTM_BF16;
+    }
+    const xlstm_status_t st =
+        check_sequence(desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in, h_out, C_out, n_out, m_out,
+                       os.h_bf16 ? 2 : 4, os.o, os.o ? (os.o_bf16 ? 2 : 4) : 0);
+    if (st != XLSTM_OK) return st;
+    FwdArgs a = pack(desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in, static_cast<float *>(h_out), C_out, n_out,
+                     m_out);
+    a.out = os;
+    return run_chunkwise(desc, a, st, workspace, workspace_bytes, stream);
 }
 
 xlstm_status_t xlstm_mlstm_fwd_recurrent(const xlstm_mlstm_desc_t *desc, const void *q,

@@ -32,6 +32,7 @@ struct ChunkP {
     const void *q, *k, *v;
     const float *ig, *fg, *C0, *n0, *m0;
     float *h, *C1, *n1, *m1;
+    OutStage out;
 };
 
 template <typename Tin, int L>
@@ -179,7 +180,7 @@ __global__ void __launch_bounds__(kThreads) chunk_simt_kernel(ChunkP p) {
                 for (int s = 0; s <= t; ++s) a += Ps[t * (L + 1) + s] * Vs[s * kDvs + r];
                 const float num = al_s[t] * Hi[x] + a;
                 const float den = fmaxf(fabsf(al_s[t] * nq_s[t] + r_s[t]), lo_s[t]);
-                if (t < len && row0 + r < dv) p.h[((size_t)bh * p.T + t0 + t) * dv + row0 + r] = num / den;
+                if (t < len && row0 + r < dv) store_h(p.out, p.h, ((size_t)bh * p.T + t0 + t) * dv + row0 + r, num / den);
             }
         }
         __syncthreads();
@@ -250,6 +251,7 @@ cudaError_t launch_chunkwise_simt(const FwdArgs &a, cudaStream_t s) {
     p.q = a.q; p.k = a.k; p.v = a.v;
     p.ig = a.ig; p.fg = a.fg; p.C0 = a.C0; p.n0 = a.n0; p.m0 = a.m0;
     p.h = a.h; p.C1 = a.C1; p.n1 = a.n1; p.m1 = a.m1;
+    p.out = a.out;
     return a.dtype == XLSTM_BF16 ? launch_typed<__nv_bfloat16>(p, s) : launch_typed<float>(p, s);
 }
 

@@ -145,6 +145,7 @@ struct TcParams {
     const float *ig, *fg, *C0, *n0, *m0;
     const float *segC, *segN, *segM;   // entry states of segments 1 .. nseg-1
     float *h, *C1, *n1, *m1;
+    OutStage out;                // h points to bf16 elements when out.h_bf16
     int32_t *status;
     int fault;
 };
@@ -276,6 +277,45 @@ __device__ __noinline__ void exact_epilogue(uint32_t tm, uint32_t lane_base, con
     }
 }
 
+// Epilogue through the output stage (an output gate, or a bf16 h): the fast and
+// the exact chunk forms with every store through store_h.  Out of line: the
+// plain fp32 epilogue stays compact.  Element (t, v) of the chunk is at
+// e0 + t * dv.
+template <class C>
+__device__ __noinline__ void gated_epilogue(uint32_t tm, uint32_t lane_base, const float *coef, const float *inv,
+                                            bool exact, size_t e0, size_t dv, int len, OutStage os, void *h) {
+#pragma unroll 1
+    for (int hh = 0; hh < 2; ++hh) {
+        float rh[32], cf[32];
+        tmem_ld32(tm + lane_base + C::TM_H + 32 * hh, rh);
+        load32(coef + 32 * hh, cf);
+        tmem_wait_ld();
+#pragma unroll
+        for (int x = 0; x < 32; ++x) rh[x] *= cf[x];
+        if (exact) {
+            float ra[32];
+            tmem_ld32(tm + lane_base + C::TM_S + 32 * hh, ra);
+            load32(inv + 32 * hh, cf);
+            tmem_wait_ld();
+#pragma unroll
+            for (int x = 0; x < 32; ++x) rh[x] = fmaf(ra[x], cf[x], rh[x]);
+        }
+        const int n = min(32, len - 32 * hh);
+        // all gate loads of the 32 tokens before any store: the stores to h could
+        // alias o~ as far as the compiler knows, and would serialise each load
+        if (os.o) {
+            float ov[32];
+#pragma unroll
+            for (int x = 0; x < 32; ++x) ov[x] = x < n ? load_o(os, e0 + (size_t)(32 * hh + x) * dv) : 0.f;
+#pragma unroll
+            for (int x = 0; x < 32; ++x) rh[x] = gate_h(rh[x], ov[x]);
+        }
+#pragma unroll
+        for (int x = 0; x < 32; ++x)
+            if (x < n) put_h(os, h, e0 + (size_t)(32 * hh + x) * dv, rh[x]);
+    }
+}
+
 // 2^e for e <= 0 with the hardware's approximate exponential (relative error far
 // below the 2^-16 of the bf16 hi/lo operands it feeds; 2^e below 2^-126 flushes to 0).
 __device__ __forceinline__ float ex2_approx(float e) {
@@ -361,7 +401,9 @@ __device__ __forceinline__ void split_range(uint32_t tm, uint32_t lane_base, int
     }
 }
 
-template <int DQK>
+// GATED: the output stage (an output gate and/or a bf16 h) is applied in the
+// epilogue; the plain instantiation keeps the fp32 store path alone.
+template <int DQK, bool GATED>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const TcParams p) {
@@ -733,6 +775,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                 coef_s[sb * kL + st] = g[kGAH + st] * inv;
             }
             named_barrier(1, 128);
+            if (GATED && alive && vok && p.out.o) {
+                // pull this chunk's o~ toward L2 while the readout MMAs run: a warp's 32
+                // rows of a token share one line, so each lane takes two tokens
+                const size_t eb = ((size_t)bh * p.T + t_base + kL * c) * p.dv + (v & ~31);
+                const int len = min(kL, T - kL * c), ln = st & 31, ob = p.out.o_bf16 ? 2 : 4;
+                const char *ob0 = static_cast<const char *>(p.out.o);
+                if (ln < len) prefetch_l2(ob0 + (eb + (size_t)ln * p.dv) * ob);
+                if (ln + 32 < len) prefetch_l2(ob0 + (eb + (size_t)(ln + 32) * p.dv) * ob);
+            }
             alive = alive && waitw(sh, &bar[B_H_FULL], c & 1, kWhereStH);
             if (alive) {
                 tc_fence_after();
@@ -749,7 +800,37 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (alive) {
                 const int len = min(kL, T - kL * c);
                 float *hc = hout + (size_t)kL * c * p.dv;
-                if (exact && vok) {
+                if (GATED && vok && exact) {
+                    gated_epilogue<C>(tm, lane_base, coef_s + sb * kL, inv_s + sb * kL, exact,
+                                      ((size_t)bh * p.T + t_base + kL * c) * p.dv + v, p.dv, len, p.out, p.h);
+                } else if (GATED && vok) {   // fast chunk through the output stage
+                    const size_t e0 = ((size_t)bh * p.T + t_base + kL * c) * p.dv + v;
+#pragma unroll 1
+                    for (int hh = 0; hh < 2; ++hh) {
+                        float rh[32], cf[32];
+                        tmem_ld32(tm + lane_base + C::TM_H + 32 * hh, rh);
+                        load32(coef_s + sb * kL + 32 * hh, cf);
+                        tmem_wait_ld();
+#pragma unroll
+                        for (int x = 0; x < 32; ++x) rh[x] *= cf[x];
+                        const int n = min(32, len - 32 * hh);
+                        const size_t e1 = e0 + (size_t)32 * hh * p.dv;
+#pragma unroll
+                        for (int q4 = 0; q4 < 2; ++q4) {   // 16 tokens at a time: gate loads first, then stores
+                            if (p.out.o) {
+                                float ov[16];
+#pragma unroll
+                                for (int i = 0; i < 16; ++i)
+                                    ov[i] = 16 * q4 + i < n ? load_o(p.out, e1 + (size_t)(16 * q4 + i) * p.dv) : 0.f;
+#pragma unroll
+                                for (int i = 0; i < 16; ++i) rh[16 * q4 + i] = gate_h(rh[16 * q4 + i], ov[i]);
+                            }
+#pragma unroll
+                            for (int i = 0; i < 16; ++i)
+                                if (16 * q4 + i < n) put_h(p.out, p.h, e1 + (size_t)(16 * q4 + i) * p.dv, rh[16 * q4 + i]);
+                        }
+                    }
+                } else if (exact && vok) {
                     exact_epilogue<C>(tm, lane_base, coef_s + sb * kL, inv_s + sb * kL, hc, p.dv, len);
                 } else if (vok) {
 #pragma unroll 1
@@ -948,6 +1029,7 @@ cudaError_t launch_dqk(const FwdArgs &a, cudaStream_t s, int fault) {
     p.T = a.T; p.dv = a.dv; p.nslices = (a.dv + kDvs - 1) / kDvs; p.scale = a.scale;
     p.ig = a.ig; p.fg = a.fg; p.C0 = a.C0; p.n0 = a.n0; p.m0 = a.m0;
     p.h = a.h; p.C1 = a.C1; p.n1 = a.n1; p.m1 = a.m1; p.status = a.status; p.fault = fault;
+    p.out = a.out;
     p.BH = BH; p.nseg = 1; p.seg_chunks = (a.T + kL - 1) / kL;
     p.segC = p.segN = p.segM = nullptr;
     cudaError_t e;
@@ -962,7 +1044,7 @@ cudaError_t launch_dqk(const FwdArgs &a, cudaStream_t s, int fault) {
             p.segM = reinterpret_cast<const float *>(ws + sp.off_M);
         }
     }
-    auto kern = chunk_tc_kernel<DQK>;
+    auto kern = (a.out.o || a.out.h_bf16) ? chunk_tc_kernel<DQK, true> : chunk_tc_kernel<DQK, false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     kern<<<BH * p.nseg * p.nslices, kThreads, C::SMEM, s>>>(tq, tk, tv, p);

@@ -8,6 +8,14 @@
 
 namespace xlstm {
 
+// Output stage (xLSTM page, "mLSTM (matrix LSTM)" eq. 3 and the o_t line of its
+// listing): h = sigmoid(o~) h~ when output-gate pre-activations are given, with
+// h stored as fp32 or bf16.  The chunkwise kernels apply it in their epilogue.
+struct OutStage {
+    const void *o = nullptr;   // [B][H][T][d_v] pre-activations o~, or null (h = h~)
+    int o_bf16 = 0, h_bf16 = 0;
+};
+
 // Everything one forward launch needs, already validated by the C ABI layer.
 struct FwdArgs {
     int B, H, T, dqk, dv;
@@ -20,6 +28,7 @@ struct FwdArgs {
     float *h, *C1, *n1, *m1;     // state outs may be null
     int32_t *status;             // device status block (4 x int32), may be null
     void *seg_ws;                // scratch for the segment-parallel chunkwise path (null: sequential)
+    OutStage out;                // chunkwise only; h points to bf16 elements when out.h_bf16
 };
 
 // How a long sequence is cut into segments that run in parallel (nseg = 1: not
@@ -46,6 +55,26 @@ void set_chunkwise_tc_fault(int mode);   // test hook: applies to the next launc
 // ---- small device helpers ------------------------------------------------
 __device__ __forceinline__ float to_f32(float x) { return x; }
 __device__ __forceinline__ float to_f32(__nv_bfloat16 x) { return __bfloat162float(x); }
+
+// Element e of o~ (read-only path).
+__device__ __forceinline__ float load_o(const OutStage &os, size_t e) {
+    return os.o_bf16 ? __bfloat162float(__ldg(static_cast<const __nv_bfloat16 *>(os.o) + e))
+                     : __ldg(static_cast<const float *>(os.o) + e);
+}
+// sigmoid(o~) h~, formed as h~ / (1 + e^{-o~}): o~ -> -inf gives a signed zero.
+__device__ __forceinline__ float gate_h(float h_tilde, float o) { return h_tilde / (1.f + expf(-o)); }
+__device__ __forceinline__ void put_h(const OutStage &os, void *h, size_t e, float val) {
+    if (os.h_bf16)
+        static_cast<__nv_bfloat16 *>(h)[e] = __float2bfloat16_rn(val);
+    else
+        static_cast<float *>(h)[e] = val;
+}
+// Pull the line holding p toward L2 (no register, no wait).
+__device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
+// Element e of h (the same flat index into o~): h~ through the output stage.
+__device__ __forceinline__ void store_h(const OutStage &os, void *h, size_t e, float h_tilde) {
+    put_h(os, h, e, os.o ? gate_h(h_tilde, load_o(os, e)) : h_tilde);
+}
 
 __device__ __forceinline__ float warp_sum(float x) {
 #pragma unroll

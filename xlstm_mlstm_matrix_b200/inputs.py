@@ -14,6 +14,9 @@ Recipe (all draws from ``numpy.random.default_rng(seed)``, in this order):
   C0, n0    normal(0, 0.1) (float32) when the workload carries an initial state
   m0        uniform(0, 5) or zero (float32)
 The decode workload draws its initial state first, then q, k, v, i~, f~ per step.
+Output-gate pre-activations o~ (the fused output stage) come from a generator of
+their own, seeded with the workload seed + 7919, so the draws above are unchanged:
+  o~        normal(0, 3) (float32), rounded to its storage dtype
 """
 from __future__ import annotations
 
@@ -148,6 +151,13 @@ def decode_steps(w: Workload, rng, n_steps: int | None = None) -> Iterator[dict]
         v = _store(rng.standard_normal((B, H, dv), dtype=np.float32), w.dtype)
         ig, fg = _gates(rng, (B, H), w)
         yield dict(q=q, k=k, v=v, i_pre=ig, f_pre=fg)
+
+
+def output_gate_pre(w: Workload, dtype: str = "bf16") -> np.ndarray:
+    """o~ [B,H,T,d_v] for the output stage, stored as dtype ("bf16" or "f32")."""
+    rng = np.random.default_rng(w.seed + 7919)
+    o = rng.standard_normal((w.B, w.H, w.T, w.d_v), dtype=np.float32) * np.float32(3.0)
+    return _store(o, dtype)
 
 
 def relative_errors(x: np.ndarray, y: np.ndarray, row_axes: int = 1):
