@@ -79,8 +79,8 @@ def test_parallel_workspace_size(lib):
         d = capi.make_desc(B, H, T, dqk, dv, dt, 1.0, L)
         assert par(d) == base(d), (B, H, T, dqk, dv, dt, L)
     assert lib.xlstm_mlstm_workspace_size_parallel(None) == 0
-    # 74 sequences fit two per SM row... two segments would be 2000 chunks long: the
-    # 1024-chunk cap makes it four segments of 1000
+    # 74 sequences on 148 SMs allow two segments each, of 2000 chunks: the 1024-chunk
+    # cap on a segment makes it four segments of 1000
     d = capi.make_desc(1, 74, 64 * 4000, 64, 128, capi.XLSTM_BF16, 1.0, 64)
     assert par(d) == base(d) + _seg_bytes(74, 4, 64, 128)
 
