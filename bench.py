@@ -148,13 +148,21 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def traffic_for(kernel_src_sha: str, workload: str):
-    """DRAM bytes per launch from the committed ncu summary, if it was taken
-    on the current kernel source for this workload; else None."""
+def traffic_for(kernel_src_sha: str, workload, gated=False):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel source for this workload at its full size (no --B/--H/--T
+    override) and on the plain output path; else None.  workload: a Workload or
+    a workload name (taken at full size)."""
+    from xlstm_mlstm_matrix_b200 import inputs
+    name = workload if isinstance(workload, str) else workload.name
+    if not isinstance(workload, str) and workload != inputs.WORKLOADS.get(name, None).replace(seed=workload.seed):
+        return None
+    if gated:
+        return None
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
-    d = json.load(open(path)).get(workload)
+    d = json.load(open(path)).get(name)
     if not d or d.get("source_sha") != kernel_src_sha:
         return None
     return d.get("traffic_bytes_per_launch")
@@ -531,7 +539,7 @@ def run_ours(args, rank, world, local_rank):
             "tflops": world * flops / (ms * 1e-3) / 1e12,
             "hbm_gbs": achieved_gbs,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved_gbs / hbm, "traffic": traffic_for(src_sha, w.name),
+                         "frac": achieved_gbs / hbm, "traffic": traffic_for(src_sha, w, gated),
                          "peak_source": peak_src, "kernel": job.kernel,
                          "algorithmic_bytes_per_launch": bytes_, "flops_per_launch": flops,
                          "tensor_frac": flops / (ms * 1e-3) / 1e12 / bf16_peak},

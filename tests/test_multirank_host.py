@@ -101,3 +101,17 @@ def test_reference_arm_under_torchrun_prints_one_line_from_rank0():
     d = json.loads(lines[0])
     assert d["impl"] == "reference" and d["n_gpus"] == 2 and d["value"] > 0
     assert d["e2e"]["h2d_bytes_per_step"] == 0 and d["cpu_baseline"]["kind"] == "oracle"
+
+
+def test_traffic_figure_only_for_the_captured_full_size_workload():
+    """roofline.traffic comes from a capture of the full-size workload on the
+    current kernel source: a smaller case of the same name, or the gated output
+    path, reports none."""
+    sha = bench.kernel_source_sha()
+    full = bench.workload_for_rank("layer_7b", 0)
+    small = bench.workload_for_rank("layer_7b", 0, T=1024)
+    other_rank = bench.workload_for_rank("layer_7b", 3)
+    assert bench.traffic_for(sha, small) is None
+    assert bench.traffic_for(sha, full, gated=True) is None
+    assert bench.traffic_for("0" * 16, full) is None
+    assert bench.traffic_for(sha, full) == bench.traffic_for(sha, other_rank)
