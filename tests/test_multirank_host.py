@@ -81,6 +81,9 @@ def test_algorithmic_bytes_match_the_counting_convention():
     b, f = bench.algorithmic(bench.workload_for_rank("layer_7b", 0))
     assert b == 1_109_459_200
     assert f == pytest.approx(150.3e9, rel=1e-3)
+    # the output stage with bf16 o~ and h: o~ read (2 B) replaces half of the fp32 h write
+    bg, fg = bench.algorithmic(bench.workload_for_rank("layer_7b", 0), gated=True)
+    assert bg == 1_109_459_200 and fg == f
     # decode step: the state is read and written once (about 1.08 GB at B=128, H=8)
     b, _ = bench.algorithmic(bench.workload_for_rank("decode", 0))
     assert b == pytest.approx(1.08e9, rel=0.01)
