@@ -8,12 +8,10 @@ each: the pins are strong enough to catch a plausible mistake anywhere.
 """
 import os
 import shutil
-import subprocess
 import tempfile
 
 import numpy as np
 import pytest
-import torch
 
 import oracle
 from oracle_pins import PINS
@@ -25,36 +23,36 @@ def test_pin(name, fn, tol):
     assert err <= tol, f"{name}: {err:.3e} > {tol:.1e}"
 
 
-def test_listing_step_agrees_when_stabilizer_stays_zero():
-    """The page's forward_recurrent listing (identity projections, o_t = 1),
-    restated in torch float64.  It carries the stabilized state but clamps
-    with 1, so it matches the stabilized readout only while m_t = 0; inputs
-    with i~ = 0 and f~ <= 0 keep m_t = 0 at every step."""
-    g = torch.Generator().manual_seed(5)
+def test_eq3_clamp_at_one_while_stabilizer_stays_zero():
+    """xLSTM page, "mLSTM (matrix LSTM)" eq. 1-3 with the "sLSTM" stabilizer.
+    With i~ = 0, f~ <= 0 and m_0 = 0 the stabilizer m_t = max(f~_t + m_{t-1}, i~_t)
+    stays 0, so the stabilized gates are the raw ones (f = e^{f~}, i = 1) and the
+    readout lower bound e^{-m_t} is the 1 of eq. 3.  Unrolling eq. 1-2 then gives
+    C_t = sum_{s<=t} e^{F_t - F_s} v_s k_s^T and n_t = sum_{s<=t} e^{F_t - F_s} k_s
+    (F_t the inclusive sum of f~), so
+      h_t = sum_s e^{F_t-F_s} (q_t.k_s) v_s / max(|sum_s e^{F_t-F_s} q_t.k_s|, 1),
+    evaluated here as one masked matrix product; the clamp is active on some
+    tokens (the small weights at the start) and inactive on others."""
+    rng = np.random.default_rng(5)
     dqk, dv, T = 6, 4, 12
-    qs = torch.randn(T, dqk, generator=g, dtype=torch.float64)
-    ks = torch.randn(T, dqk, generator=g, dtype=torch.float64)
-    vs = torch.randn(T, dv, generator=g, dtype=torch.float64)
-    fs = -torch.rand(T, generator=g, dtype=torch.float64)
-    its = torch.zeros(T, dtype=torch.float64)
-    C = torch.zeros(dv, dqk, dtype=torch.float64)
-    n = torch.zeros(dqk, dtype=torch.float64)
-    m = torch.zeros((), dtype=torch.float64)
-    hs = []
-    for t in range(T):
-        m_t = torch.max(fs[t] + m, its[t])
-        f_t = torch.exp(fs[t] + m - m_t)
-        i_t = torch.exp(its[t] - m_t)
-        C = f_t * C + i_t * torch.outer(vs[t], ks[t])
-        n = f_t * n + i_t * ks[t]
-        hs.append((C @ qs[t]) / torch.clamp(torch.abs(n @ qs[t]), min=1.0))
-        m = m_t
-    h, Co, no, mo = oracle.forward(qs.numpy()[None, None], ks.numpy()[None, None],
-                                   vs.numpy()[None, None], its.numpy()[None, None],
-                                   fs.numpy()[None, None])
-    assert np.max(np.abs(h[0, 0] - torch.stack(hs).numpy())) < 1e-13
-    assert np.max(np.abs(Co[0, 0] - C.numpy())) < 1e-13
-    assert abs(mo[0, 0]) == 0.0
+    q = rng.standard_normal((T, dqk))
+    k = rng.standard_normal((T, dqk))
+    v = rng.standard_normal((T, dv))
+    f = -rng.uniform(0.0, 1.0, T)
+    i = np.zeros(T)
+    F = np.cumsum(f)
+    decay = np.tril(np.exp(F[:, None] - F[None, :]))
+    A = (q @ k.T) * decay
+    den = np.abs(A.sum(axis=1))
+    assert np.any(den < 1.0) and np.any(den > 1.0), "both sides of the clamp must be exercised"
+    h_closed = (A @ v) / np.maximum(den, 1.0)[:, None]
+    C_closed = (v * np.exp(F[-1] - F)[:, None]).T @ k
+    n_closed = np.exp(F[-1] - F) @ k
+    h, C, n, m = oracle.forward(q[None, None], k[None, None], v[None, None], i[None, None], f[None, None])
+    assert np.max(np.abs(h[0, 0] - h_closed)) < 1e-13
+    assert np.max(np.abs(C[0, 0] - C_closed)) < 1e-13
+    assert np.max(np.abs(n[0, 0] - n_closed)) < 1e-13
+    assert m[0, 0] == 0.0
 
 
 def test_empty_and_degenerate_shapes():
