@@ -553,6 +553,59 @@ def run_ours(args, rank, world, local_rank):
         print(json.dumps(line), flush=True)
 
 
+def run_mma_probe():
+    """tcgen05.mma issue cost: one thread issues back-to-back MMAs (K = 16, bf16
+    operands, zero data) and clock64 brackets the sequence up to the completion
+    of a final commit.  Prints one table row per shape: cycles per instruction
+    on one CTA and the median over 148 CTAs (one per SM), and the fraction of
+    the tensor pipe's dense rate that cost implies (M = 128: 8192 flop per SM
+    cycle; M = 64 runs on half the datapath)."""
+    import ctypes
+    import torch  # noqa: F401  (CUDA context for the probe library)
+    lib = ctypes.CDLL(os.path.join(ROOT, "xlstm_mlstm_matrix_b200", "libxlstm_mma_probe.so"))
+    f = lib.mma_probe_run
+    f.restype = ctypes.c_int
+    f.argtypes = [ctypes.c_int] * 10 + [ctypes.POINTER(ctypes.c_longlong)]
+    issue_names = {0: "one thread", 1: "warp + elect.sync", 2: "two warps", 3: "one thread, unrolled",
+                   4: "rolled K loop", 5: "unrolled, integer op between", 6: "unrolled, runtime base",
+                   7: "unrolled by 4", 8: "no MMA", 9: "one thread, unrolled (ts)"}
+    bg_names = {0: "", 1: " + bg tmem ld", 2: " + bg tmem st", 3: " + bg smem ld", 4: " + bg smem st"}
+    cases = []   # (form, M, N, a_mn, b_mn, accumulators, commit_every, issue + 16 * background)
+    for M, N in ((64, 64), (128, 64), (128, 128), (128, 256)):
+        cases.append(("ss", M, N, 0, 0, 1, 0, 0))
+    cases += [("ts", 128, 64, 0, 0, 1, 0, 0), ("ss", 128, 64, 1, 1, 1, 0, 0), ("ss", 128, 64, 0, 0, 2, 0, 0),
+              ("ss", 128, 64, 0, 0, 1, 1, 0), ("ss", 128, 64, 0, 0, 1, 0, 1), ("ss", 128, 64, 0, 0, 1, 0, 2),
+              ("ss", 128, 64, 0, 0, 1, 0, 4), ("ss", 128, 64, 0, 0, 1, 0, 5), ("ss", 128, 64, 0, 0, 1, 0, 6),
+              ("ss", 128, 64, 0, 0, 1, 0, 7)]
+    for M, N in ((64, 64), (128, 64), (128, 128), (128, 256)):
+        cases.append(("ss", M, N, 0, 0, 1, 0, 3))
+    for N in (64, 128, 256):
+        cases.append(("ts", 128, N, 0, 0, 1, 0, 9))
+    # background traffic on warps 1-3: alone, and beside unrolled MMAs
+    for bg in (1, 2, 3, 4):
+        cases += [("ss", 128, 64, 0, 0, 1, 0, 8 + 16 * bg), ("ss", 128, 64, 0, 0, 1, 0, 3 + 16 * bg),
+                  ("ts", 128, 64, 0, 0, 1, 0, 9 + 16 * bg), ("ss", 128, 256, 0, 0, 1, 0, 3 + 16 * bg)]
+    nmma = 512
+    for form, M, N, amn, bmn, nacc, ce, issue in cases:
+        res, bgc = {}, {}
+        for ctas in (1, 148):
+            buf = (ctypes.c_longlong * (3 * ctas))()
+            rc = f(1 if form == "ts" else 0, M, N, amn, bmn, nmma, nacc, ce, issue, ctas, buf)
+            if rc != 0:
+                raise SystemExit(f"probe failed rc={rc} for {form} M{M} N{N} issue {issue}")
+            vals = list(buf)
+            res[ctas] = statistics.median(vals[:ctas]) / nmma
+            its = vals[ctas:2 * ctas]
+            bgc[ctas] = statistics.median([c / i for c, i in zip(vals[2 * ctas:], its) if i > 0]) if any(its) else None
+        ideal = M * N * 16 * 2 / (8192 if M == 128 else 4096)
+        row = {"form": form, "M": M, "N": N, "a_mn": amn, "b_mn": bmn, "accumulators": nacc,
+               "commit_every": ce, "issue": issue_names[issue % 16] + bg_names[issue // 16],
+               "cycles_1cta": round(res[1], 1), "cycles_148cta": round(res[148], 1), "ideal_cycles": ideal,
+               "pipe_frac_148": round(ideal / res[148], 3) if res[148] else None,
+               "bg_cycles_per_iter_148": None if bgc[148] is None else round(bgc[148], 1)}
+        print(json.dumps(row), flush=True)
+
+
 def main():
     from xlstm_mlstm_matrix_b200.inputs import WORKLOADS
     ap = argparse.ArgumentParser()
@@ -570,7 +623,12 @@ def main():
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
     ap.add_argument("--H", type=int, default=0, help="override the head count (profiling)")
     ap.add_argument("--T", type=int, default=0, help="override the sequence length (profiling)")
+    ap.add_argument("--probe", choices=["mma"], default=None,
+                    help="mma: tcgen05.mma issue-cost microbenchmark instead of the benchmark")
     args = ap.parse_args()
+    if args.probe == "mma":
+        run_mma_probe()
+        return
     args.warmup = max(3, args.warmup)
     rank = int(os.environ.get("RANK", 0))
     world = int(os.environ.get("WORLD_SIZE", 1))

@@ -18,6 +18,9 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 OUT = os.path.join(HERE, "libxlstm_mlstm.so")
+# tcgen05 issue-cost microbenchmark (measurement tooling, driven by bench.py --probe mma)
+PROBE_SRC = os.path.join(CSRC, "probe", "mma_cost.cu")
+PROBE_OUT = os.path.join(HERE, "libxlstm_mma_probe.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
@@ -65,6 +68,10 @@ def build(verbose: bool = False, extra=()) -> str:
     tmp = OUT + f".tmp{os.getpid()}"
     subprocess.check_call([nvcc(), "-shared", "-o", tmp] + objs + ARCH)
     os.replace(tmp, OUT)
+    probe = _compile(PROBE_SRC, extra)
+    tmp = PROBE_OUT + f".tmp{os.getpid()}"
+    subprocess.check_call([nvcc(), "-shared", "-o", tmp, probe] + ARCH)
+    os.replace(tmp, PROBE_OUT)
     if verbose:
         print(OUT)
     return OUT
