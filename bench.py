@@ -568,8 +568,10 @@ def run_mma_probe():
     f.argtypes = [ctypes.c_int] * 10 + [ctypes.POINTER(ctypes.c_longlong)]
     issue_names = {0: "one thread", 1: "warp + elect.sync", 2: "two warps", 3: "one thread, unrolled",
                    4: "rolled K loop", 5: "unrolled, integer op between", 6: "unrolled, runtime base",
-                   7: "unrolled by 4", 8: "no MMA", 9: "one thread, unrolled (ts)"}
-    bg_names = {0: "", 1: " + bg tmem ld", 2: " + bg tmem st", 3: " + bg smem ld", 4: " + bg smem st"}
+                   7: "unrolled by 4", 8: "no MMA", 9: "one thread, unrolled (ts)",
+                   10: "chunk program, rolled", 11: "chunk program, unrolled"}
+    bg_names = {0: "", 1: " + bg tmem ld", 2: " + bg tmem st", 3: " + bg smem ld", 4: " + bg smem st",
+                5: " + bg alu", 6: " + bg bulk copies"}
     cases = []   # (form, M, N, a_mn, b_mn, accumulators, commit_every, issue + 16 * background)
     for M, N in ((64, 64), (128, 64), (128, 128), (128, 256)):
         cases.append(("ss", M, N, 0, 0, 1, 0, 0))
@@ -585,8 +587,25 @@ def run_mma_probe():
     for bg in (1, 2, 3, 4):
         cases += [("ss", 128, 64, 0, 0, 1, 0, 8 + 16 * bg), ("ss", 128, 64, 0, 0, 1, 0, 3 + 16 * bg),
                   ("ts", 128, 64, 0, 0, 1, 0, 9 + 16 * bg), ("ss", 128, 256, 0, 0, 1, 0, 3 + 16 * bg)]
+    # pseudo-random operands (+256), and background traffic on 11 warps (+128)
+    R, W = 256, 128
+    cases += [("ss", 64, 64, 0, 0, 1, 0, 3 + R), ("ss", 128, 64, 0, 0, 1, 0, 3 + R), ("ss", 128, 128, 0, 0, 1, 0, 3 + R),
+              ("ss", 128, 256, 0, 0, 1, 0, 3 + R), ("ts", 128, 64, 0, 0, 1, 0, 9 + R), ("ts", 128, 256, 0, 0, 1, 0, 9 + R),
+              ("ss", 128, 64, 0, 0, 1, 0, 4 + R)]
+    for bg in (1, 2, 3, 4):
+        cases += [("ss", 128, 64, 0, 0, 1, 0, 8 + 16 * bg + W + R), ("ss", 128, 64, 0, 0, 1, 0, 3 + 16 * bg + W + R),
+                  ("ts", 128, 64, 0, 0, 1, 0, 9 + 16 * bg + W + R)]
+    # the chunkwise kernel's per-chunk MMA program (56 MMAs + 6 commits), alone and beside busy warps
+    for prog in (10, 11):
+        cases += [("ss", 128, 64, 0, 0, 1, 0, prog), ("ss", 128, 64, 0, 0, 1, 0, prog + 16 * 5 + W),
+                  ("ss", 128, 64, 0, 0, 1, 0, prog + 16 * 3 + W), ("ss", 128, 64, 0, 0, 1, 0, prog + 16 * 1 + W),
+                  ("ss", 128, 64, 0, 0, 1, 0, prog + 16 * 6)]
+    cases += [("ss", 128, 64, 0, 0, 1, 0, 8 + 16 * 6), ("ss", 128, 64, 0, 0, 1, 0, 3 + 16 * 6),
+              ("ts", 128, 64, 0, 0, 1, 0, 9 + 16 * 6)]
     nmma = 512
     for form, M, N, amn, bmn, nacc, ce, issue in cases:
+        if issue % 16 >= 10:
+            nmma = 56 * 32
         res, bgc = {}, {}
         for ctas in (1, 148):
             buf = (ctypes.c_longlong * (3 * ctas))()
@@ -599,11 +618,15 @@ def run_mma_probe():
             bgc[ctas] = statistics.median([c / i for c, i in zip(vals[2 * ctas:], its) if i > 0]) if any(its) else None
         ideal = M * N * 16 * 2 / (8192 if M == 128 else 4096)
         row = {"form": form, "M": M, "N": N, "a_mn": amn, "b_mn": bmn, "accumulators": nacc,
-               "commit_every": ce, "issue": issue_names[issue % 16] + bg_names[issue // 16],
+               "commit_every": ce, "issue": issue_names[issue % 16] + bg_names[(issue // 16) % 8] +
+               (" x11 warps" if issue & 128 else "") + (", random data" if issue & 256 else ""),
                "cycles_1cta": round(res[1], 1), "cycles_148cta": round(res[148], 1), "ideal_cycles": ideal,
                "pipe_frac_148": round(ideal / res[148], 3) if res[148] else None,
                "bg_cycles_per_iter_148": None if bgc[148] is None else round(bgc[148], 1)}
+        if issue % 16 >= 10:
+            row["cycles_per_chunk_148"] = round(res[148] * nmma / 32)
         print(json.dumps(row), flush=True)
+        nmma = 512
 
 
 def main():

@@ -43,8 +43,8 @@
 //
 // Warps: 0 TMA producer (and L2 prefetch two chunks ahead), 1 MMA issuer (owns
 // TMEM), 2 gate scan, 3 normaliser,
-// 4-7 state group (the first columns of the state split, epilogue), 8-11 token
-// group (w V, the other columns of the state split, n.q, P).
+// 4-7 state group (the first columns of the state split, n.q, epilogue), 8-11
+// token group (w V, the other columns of the state split, P).
 // Every wait is bounded: one that gives up records XLSTM_ERR_TIMEOUT in the
 // status block; each role drains what it has in flight, TMEM is freed, return.
 #include <math.h>
@@ -72,7 +72,8 @@ enum : int32_t {
     kWhereTmaKvEmpty = 1, kWhereTmaQEmpty, kWhereMmaKvFull, kWhereMmaQFull, kWhereMmaSEmpty, kWhereMmaGate,
     kWhereMmaConv, kWhereMmaOps, kWhereMmaVt, kWhereMmaHEmpty, kWhereMmaClo, kWhereGateEmpty, kWhereNormGate,
     kWhereNormKv, kWhereNormFree, kWhereStUpd, kWhereStGate, kWhereStClo, kWhereStOps, kWhereStH, kWhereStFinal,
-    kWhereTkH, kWhereTkGate, kWhereTkKv, kWhereTkQ, kWhereTkN, kWhereTkS, kWhereTkUpd, kWhereTkClo, kWhereTkConv
+    kWhereTkH, kWhereTkGate, kWhereTkKv, kWhereTkQ, kWhereTkN, kWhereTkS, kWhereTkUpd, kWhereTkClo, kWhereTkConv,
+    kWhereStQ, kWhereStN
 };
 
 // Test hook: make the gate warp withhold one hand-off so that its consumers time out.
@@ -381,6 +382,41 @@ __device__ __noinline__ void exact_p_pass(uint32_t s_tmem, const float *g, uint8
         rsum += r0[i];
     }
     store_p_row(r0, Ps, rs, rsum, t, lane);
+}
+
+// n.q_t of one chunk in fp32: two threads per token (trow), each over half of
+// d_qk, the halves joined by a lane shuffle; stores AN_t (n_acc . q_t).
+template <class C>
+__device__ __forceinline__ void nq_pass(const uint8_t *Qs, const float *nbuf_s, const float *g, float *nq, int trow,
+                                        int half) {
+    constexpr int DQK = C::NKB * 64;
+    const float *nn = nbuf_s + (half ? 4 : 0);
+    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+#pragma unroll 1
+    for (int g0 = 0; g0 < DQK / 16; g0 += 4) {
+        uint4 u[4];
+        float4 na[4], nb[4];
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+            // the upper-half thread walks its chunks rotated by 4 so that the
+            // pair of a token hits distinct banks
+            const int ci = half ? (g0 + k4 + 4) % (DQK / 16) : g0 + k4;
+            const int jc = half * (DQK / 2) + 8 * ci;
+            u[k4] = *reinterpret_cast<const uint4 *>(Qs + (jc >> 6) * 8192 + sw128_offset(trow, (jc & 63) >> 3));
+            na[k4] = *reinterpret_cast<const float4 *>(nn + jc);
+            nb[k4] = *reinterpret_cast<const float4 *>(nn + jc + 4);
+        }
+#pragma unroll
+        for (int k4 = 0; k4 < 4; ++k4) {
+            acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].x), make_float2(na[k4].x, na[k4].y), acc[k4]);
+            acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].y), make_float2(na[k4].z, na[k4].w), acc[k4]);
+            acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].z), make_float2(nb[k4].x, nb[k4].y), acc[k4]);
+            acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].w), make_float2(nb[k4].z, nb[k4].w), acc[k4]);
+        }
+    }
+    float v = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) + ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
+    v += __shfl_xor_sync(0xffffffffu, v, 1);
+    if (half == 0) nq[trow] = g[kGAN + trow] * v;
 }
 
 // Blocks [i0, i1) of this thread's C_acc row through split_state_block, with the
@@ -767,7 +803,17 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             named_barrier(1, 128);
             if (st == 0 && alive) mbar_arrive(&bar[B_CONV0]);
-            // --- denominators, once the token group has published n.q and the row sums
+            // --- n.q_t of this chunk (coefficient AN_t = scale e^{b - mu_t}); the state group
+            //     waits for the readout anyway, so it takes this off the token group
+            alive = alive && waitw(sh, &bar[B_Q_FULL + s], (c >> 1) & 1, kWhereStQ);
+            alive = alive && waitw(sh, &bar[B_N_READY + s], (c >> 1) & 1, kWhereStN);
+            if (alive) nq_pass<C>(sm + C::OFF_Q + s * C::Q_BYTES, nbuf + s * C::NBUF, g, nq_s + sb * kL, st >> 1, st & 1);
+            named_barrier(1, 128);
+            if (st == 0 && alive) {
+                mbar_arrive(&bar[B_Q_EMPTY + s]);
+                mbar_arrive(&bar[B_N_FREE + s]);
+            }
+            // --- denominators, once the token group has published the row sums
             alive = alive && waitw(sh, &bar[B_OPS], c & 1, kWhereStOps);
             if (alive && st < kL) {
                 const float inv = 1.f / fmaxf(fabsf(nq_s[sb * kL + st] + rs_s[sb * kL + st]), g[kGLower + st]);
@@ -888,12 +934,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tk = tid - 256;            // 0..127
         const int wq = warp - 8;             // TMEM lane quarter
         const uint32_t lane_base = (uint32_t)(32 * wq) << 16;
-        const int trow = tk >> 1, half = tk & 1;     // n.q pass: token row, half of d_qk
         uint8_t *clo_s = sm + C::OFF_CLO;
         bool alive = true;
-        // Chunk c-1 in the loop body below, then the operands of chunk c that need
-        // neither its split nor the P tile: V(c) <- w V(c) (fast chunks) and n.q_t.
-        // They overlap the readout MMAs of chunk c-1 instead of following them.
+        // Chunk c-1 in the loop body below, then the operand of chunk c that needs
+        // neither its split nor the P tile: V(c) <- w V(c) (fast chunks).  It
+        // overlaps the readout MMAs of chunk c-1 instead of following them.
         for (int c = -1; c < NC; ++c) {
           if (c >= 0) {
             const int slot = c % kNG, sb = c & 1;
@@ -952,7 +997,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (c + 1 < NC) {
                 const int j = c + 1, sj = j & 1, slot_j = j % kNG;
                 const float *gj = gring + slot_j * C::G_FLOATS;
-                // the state group has read the n.q slot of chunk j-2 (its split of chunk c follows)
+                // the MMA warp waits for w V(c) right after the split of chunk c: scaling V(c+1)
+                // only after that split keeps the two phases of B_VT from both completing
+                // before the MMA warp has waited for the first
                 if (c >= 0) alive = alive && waitw(sh, &bar[B_CONV0], c & 1, kWhereTkConv);
                 alive = alive && waitw(sh, &bar[B_G_FULL + slot_j], (j / kNG) & 1, kWhereTkGate);
                 const bool ex = alive && gj[kGScal + kSExact] != 0.f;
@@ -964,47 +1011,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
                 named_barrier(2, 128);   // unconditional: every warp of the group takes every barrier
                 if (tk == 0 && alive && !ex) mbar_arrive(&bar[B_VT]);
-                // --- n.q_t in fp32 (coefficient AN_t = scale e^{b - mu_t})
-                alive = alive && waitw(sh, &bar[B_Q_FULL + sj], (j >> 1) & 1, kWhereTkQ);
-                alive = alive && waitw(sh, &bar[B_N_READY + sj], (j >> 1) & 1, kWhereTkN);
-                if (alive) {
-                    const uint8_t *Qs = sm + C::OFF_Q + sj * C::Q_BYTES;
-                    const float *nn = nbuf + sj * C::NBUF + (half ? 4 : 0);
-                    float2 acc[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f),
-                                     make_float2(0.f, 0.f)};
-#pragma unroll 1
-                    for (int g0 = 0; g0 < DQK / 16; g0 += 4) {
-                        uint4 u[4];
-                        float4 na[4], nb[4];
-#pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4) {
-                            // the upper-half thread walks its chunks rotated by 4 so that the
-                            // pair of a token hits distinct banks
-                            const int ci = half ? (g0 + k4 + 4) % (DQK / 16) : g0 + k4;
-                            const int jc = half * (DQK / 2) + 8 * ci;
-                            u[k4] = *reinterpret_cast<const uint4 *>(Qs + (jc >> 6) * 8192 +
-                                                                       sw128_offset(trow, (jc & 63) >> 3));
-                            na[k4] = *reinterpret_cast<const float4 *>(nn + jc);
-                            nb[k4] = *reinterpret_cast<const float4 *>(nn + jc + 4);
-                        }
-#pragma unroll
-                        for (int k4 = 0; k4 < 4; ++k4) {
-                            acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].x), make_float2(na[k4].x, na[k4].y), acc[k4]);
-                            acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].y), make_float2(na[k4].z, na[k4].w), acc[k4]);
-                            acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].z), make_float2(nb[k4].x, nb[k4].y), acc[k4]);
-                            acc[k4] = __ffma2_rn(bf16x2_to_float2(u[k4].w), make_float2(nb[k4].z, nb[k4].w), acc[k4]);
-                        }
-                    }
-                    float nq = ((acc[0].x + acc[0].y) + (acc[1].x + acc[1].y)) +
-                               ((acc[2].x + acc[2].y) + (acc[3].x + acc[3].y));
-                    nq += __shfl_xor_sync(0xffffffffu, nq, 1);
-                    if (half == 0) nq_s[sj * kL + trow] = gj[kGAN + trow] * nq;
-                }
-                named_barrier(2, 128);
-                if (tk == 0 && alive) {
-                    mbar_arrive(&bar[B_Q_EMPTY + sj]);
-                    mbar_arrive(&bar[B_N_FREE + sj]);
-                }
             }
             if (c == -1) named_barrier(3, 256);   // C_acc is initialised before either group splits it
         }
