@@ -309,7 +309,7 @@ def run_reference(args, rank, world):
 
 class _Sequence:
     """One chunkwise forward over the whole batch per step (gated: through the
-    fused output stage, bf16 o~ in and bf16 h out)."""
+    output stage, bf16 o~ in and bf16 h out)."""
 
     def __init__(self, w, inp, dev, stream, gated=False):
         import torch
@@ -348,7 +348,10 @@ class _Sequence:
                          P(self.ws), wsb, ctypes.c_void_p(stream.cuda_stream))
         self.stream = stream
         self.kernel = "chunkwise (segment summaries + combine + chunkwise)" if segmented else "chunkwise"
-        self.launches = 3 if segmented else 1   # kernels per call
+        # kernels per call: the tensor-core path applies the output gate as a second, streaming pass
+        self.launches = (3 if segmented else 1) + (1 if gated else 0)
+        if gated:
+            self.kernel += " + output gate"
         self.name = "xlstm_mlstm_fwd_chunkwise_out" if gated else "xlstm_mlstm_fwd_chunkwise"
 
     def step(self, i):

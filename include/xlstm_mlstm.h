@@ -130,13 +130,16 @@ typedef struct {
 } xlstm_mlstm_output_t;
 
 /*
- * xlstm_mlstm_fwd_chunkwise with the output stage fused into the epilogue:
+ * xlstm_mlstm_fwd_chunkwise with the output stage:
  * h_out[b][h][t][:] = sigmoid(o_pre[b][h][t][:]) * h~_t (elementwise), stored as
  * out->h_dtype.  out == NULL is xlstm_mlstm_fwd_chunkwise exactly.  Same
  * arguments, rules, workspace and status block otherwise; h_out holds
  * B*H*T*d_v elements of h_dtype.  Invalid dtypes or a misaligned o_pre give
  * XLSTM_ERR_INVALID_ARG.  The state outputs are the recurrence's, untouched by
- * the gate.
+ * the gate.  On the tensor-core path the chunkwise kernel stores h~ in h_dtype
+ * and a second, streaming kernel on the same stream applies the gate in place
+ * (with a bf16 h, h~ is rounded to bf16 before the gate and the gated value
+ * again); on the fp32 CUDA-core path the gate is applied in the epilogue.
  */
 XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise_out(
     const xlstm_mlstm_desc_t *desc, const xlstm_mlstm_output_t *out,

@@ -1,4 +1,4 @@
-"""The output stage fused into the chunkwise epilogue, against the oracle.
+"""The output stage of the chunkwise call, against the oracle.
 
 xlstm_mlstm_fwd_chunkwise_out applies h = sigmoid(o~) h~ (xLSTM page,
 "mLSTM (matrix LSTM)" eq. 3, with o_t = sigmoid(o~_t) as in the page's

@@ -149,7 +149,6 @@ struct TcParams {
     const float *ig, *fg, *C0, *n0, *m0;
     const float *segC, *segN, *segM;   // entry states of segments 1 .. nseg-1
     float *h, *C1, *n1, *m1;
-    OutStage out;                // h points to bf16 elements when out.h_bf16
     int32_t *status;
     int fault;
 };
@@ -281,13 +280,13 @@ __device__ __noinline__ void exact_epilogue(uint32_t tm, uint32_t lane_base, con
     }
 }
 
-// Epilogue through the output stage (an output gate, or a bf16 h): the fast and
-// the exact chunk forms with every store through store_h.  Out of line: the
-// plain fp32 epilogue stays compact.  Element (t, v) of the chunk is at
-// e0 + t * dv.
+// Epilogue of a chunk stored as bf16 h~ (the output stage's bf16 h; the output
+// gate, if any, is applied by a separate pass): the fast and the exact chunk
+// forms.  Out of line: the plain fp32 epilogue stays compact.  Element (t, v)
+// of the chunk is at h + t * dv.
 template <class C>
-__device__ __noinline__ void gated_epilogue(uint32_t tm, uint32_t lane_base, const float *coef, const float *inv,
-                                            bool exact, size_t e0, size_t dv, int len, OutStage os, void *h) {
+__device__ __noinline__ void bf16_epilogue(uint32_t tm, uint32_t lane_base, const float *coef, const float *inv,
+                                           bool exact, __nv_bfloat16 *h, size_t dv, int len) {
 #pragma unroll 1
     for (int hh = 0; hh < 2; ++hh) {
         float rh[32], cf[32];
@@ -305,18 +304,10 @@ __device__ __noinline__ void gated_epilogue(uint32_t tm, uint32_t lane_base, con
             for (int x = 0; x < 32; ++x) rh[x] = fmaf(ra[x], cf[x], rh[x]);
         }
         const int n = min(32, len - 32 * hh);
-        // all gate loads of the 32 tokens before any store: the stores to h could
-        // alias o~ as far as the compiler knows, and would serialise each load
-        if (os.o) {
-            float ov[32];
-#pragma unroll
-            for (int x = 0; x < 32; ++x) ov[x] = x < n ? load_o(os, e0 + (size_t)(32 * hh + x) * dv) : 0.f;
-#pragma unroll
-            for (int x = 0; x < 32; ++x) rh[x] = gate_h(rh[x], ov[x]);
-        }
+        __nv_bfloat16 *hrow = h + (size_t)32 * hh * dv;
 #pragma unroll
         for (int x = 0; x < 32; ++x)
-            if (x < n) put_h(os, h, e0 + (size_t)(32 * hh + x) * dv, rh[x]);
+            if (x < n) hrow[(size_t)x * dv] = __float2bfloat16_rn(rh[x]);
     }
 }
 
@@ -439,9 +430,9 @@ __device__ __forceinline__ void split_range(uint32_t tm, uint32_t lane_base, int
     }
 }
 
-// GATED: the output stage (an output gate and/or a bf16 h) is applied in the
-// epilogue; the plain instantiation keeps the fp32 store path alone.
-template <int DQK, bool GATED>
+// BF16H: h~ is stored as bf16 (the output stage's bf16 h); the plain
+// instantiation keeps the fp32 store path alone.
+template <int DQK, bool BF16H>
 __global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const TcParams p) {
@@ -821,15 +812,6 @@ __global__ void __launch_bounds__(kThreads, 1)
                 coef_s[sb * kL + st] = g[kGAH + st] * inv;
             }
             named_barrier(1, 128);
-            if (GATED && alive && vok && p.out.o) {
-                // pull this chunk's o~ toward L2 while the readout MMAs run: a warp's 32
-                // rows of a token share one line, so each lane takes two tokens
-                const size_t eb = ((size_t)bh * p.T + t_base + kL * c) * p.dv + (v & ~31);
-                const int len = min(kL, T - kL * c), ln = st & 31, ob = p.out.o_bf16 ? 2 : 4;
-                const char *ob0 = static_cast<const char *>(p.out.o);
-                if (ln < len) prefetch_l2(ob0 + (eb + (size_t)ln * p.dv) * ob);
-                if (ln + 32 < len) prefetch_l2(ob0 + (eb + (size_t)(ln + 32) * p.dv) * ob);
-            }
             alive = alive && waitw(sh, &bar[B_H_FULL], c & 1, kWhereStH);
             if (alive) {
                 tc_fence_after();
@@ -846,36 +828,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (alive) {
                 const int len = min(kL, T - kL * c);
                 float *hc = hout + (size_t)kL * c * p.dv;
-                if (GATED && vok && exact) {
-                    gated_epilogue<C>(tm, lane_base, coef_s + sb * kL, inv_s + sb * kL, exact,
-                                      ((size_t)bh * p.T + t_base + kL * c) * p.dv + v, p.dv, len, p.out, p.h);
-                } else if (GATED && vok) {   // fast chunk through the output stage
-                    const size_t e0 = ((size_t)bh * p.T + t_base + kL * c) * p.dv + v;
-#pragma unroll 1
-                    for (int hh = 0; hh < 2; ++hh) {
-                        float rh[32], cf[32];
-                        tmem_ld32(tm + lane_base + C::TM_H + 32 * hh, rh);
-                        load32(coef_s + sb * kL + 32 * hh, cf);
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int x = 0; x < 32; ++x) rh[x] *= cf[x];
-                        const int n = min(32, len - 32 * hh);
-                        const size_t e1 = e0 + (size_t)32 * hh * p.dv;
-#pragma unroll
-                        for (int q4 = 0; q4 < 2; ++q4) {   // 16 tokens at a time: gate loads first, then stores
-                            if (p.out.o) {
-                                float ov[16];
-#pragma unroll
-                                for (int i = 0; i < 16; ++i)
-                                    ov[i] = 16 * q4 + i < n ? load_o(p.out, e1 + (size_t)(16 * q4 + i) * p.dv) : 0.f;
-#pragma unroll
-                                for (int i = 0; i < 16; ++i) rh[16 * q4 + i] = gate_h(rh[16 * q4 + i], ov[i]);
-                            }
-#pragma unroll
-                            for (int i = 0; i < 16; ++i)
-                                if (16 * q4 + i < n) put_h(p.out, p.h, e1 + (size_t)(16 * q4 + i) * p.dv, rh[16 * q4 + i]);
-                        }
-                    }
+                if (BF16H && vok) {
+                    bf16_epilogue<C>(tm, lane_base, coef_s + sb * kL, inv_s + sb * kL, exact,
+                                     static_cast<__nv_bfloat16 *>(static_cast<void *>(p.h)) +
+                                         ((size_t)bh * p.T + t_base + kL * c) * p.dv + v,
+                                     p.dv, len);
                 } else if (exact && vok) {
                     exact_epilogue<C>(tm, lane_base, coef_s + sb * kL, inv_s + sb * kL, hc, p.dv, len);
                 } else if (vok) {
@@ -1035,7 +992,6 @@ cudaError_t launch_dqk(const FwdArgs &a, cudaStream_t s, int fault) {
     p.T = a.T; p.dv = a.dv; p.nslices = (a.dv + kDvs - 1) / kDvs; p.scale = a.scale;
     p.ig = a.ig; p.fg = a.fg; p.C0 = a.C0; p.n0 = a.n0; p.m0 = a.m0;
     p.h = a.h; p.C1 = a.C1; p.n1 = a.n1; p.m1 = a.m1; p.status = a.status; p.fault = fault;
-    p.out = a.out;
     p.BH = BH; p.nseg = 1; p.seg_chunks = (a.T + kL - 1) / kL;
     p.segC = p.segN = p.segM = nullptr;
     cudaError_t e;
@@ -1050,11 +1006,14 @@ cudaError_t launch_dqk(const FwdArgs &a, cudaStream_t s, int fault) {
             p.segM = reinterpret_cast<const float *>(ws + sp.off_M);
         }
     }
-    auto kern = (a.out.o || a.out.h_bf16) ? chunk_tc_kernel<DQK, true> : chunk_tc_kernel<DQK, false>;
+    auto kern = a.out.h_bf16 ? chunk_tc_kernel<DQK, true> : chunk_tc_kernel<DQK, false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
     kern<<<BH * p.nseg * p.nslices, kThreads, C::SMEM, s>>>(tq, tk, tv, p);
-    return cudaGetLastError();
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    // the output gate as one streaming pass over h~ in place
+    if (a.out.o) return launch_output_gate(a.out, a.h, (size_t)BH * a.T * a.dv, s);
+    return cudaSuccess;
 }
 
 }  // namespace

@@ -50,6 +50,8 @@ cudaError_t launch_chunkwise_simt(const FwdArgs &a, cudaStream_t s);
 bool chunkwise_tc_shape_ok(const FwdArgs &a);     // shapes the tensor-core kernel takes
 bool chunkwise_tc_supported(const FwdArgs &a);    // ... and the driver's TMA encoder is available
 cudaError_t launch_chunkwise_tc(const FwdArgs &a, cudaStream_t s);
+// h <- sigmoid(o~) h~ over n elements in place (h in the output stage's dtype).
+cudaError_t launch_output_gate(const OutStage &os, void *h, size_t n, cudaStream_t s);
 void set_chunkwise_tc_fault(int mode);   // test hook: applies to the next launch only
 
 // ---- small device helpers ------------------------------------------------
@@ -69,8 +71,6 @@ __device__ __forceinline__ void put_h(const OutStage &os, void *h, size_t e, flo
     else
         static_cast<float *>(h)[e] = val;
 }
-// Pull the line holding p toward L2 (no register, no wait).
-__device__ __forceinline__ void prefetch_l2(const void *p) { asm volatile("prefetch.global.L2 [%0];" ::"l"(p)); }
 // Element e of h (the same flat index into o~): h~ through the output stage.
 __device__ __forceinline__ void store_h(const OutStage &os, void *h, size_t e, float h_tilde) {
     put_h(os, h, e, os.o ? gate_h(h_tilde, load_o(os, e)) : h_tilde);
