@@ -434,6 +434,63 @@ class _Decode:
         return pairs_in, pairs_out
 
 
+def time_job(job, steps, warmup, stream, dev, gpu_index):
+    """Warm-up, then `steps` launches bracketed by CUDA events on the launch
+    stream with clock samples during the timed region: (ms per step, clocks)."""
+    import torch
+    with torch.cuda.stream(stream):
+        for i in range(warmup):
+            job.step(i)
+    stream.synchronize()
+    job.check_status()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    with ClockSampler(gpu_index) as clk:
+        clk.mark(True)
+        e0.record(stream)
+        for i in range(steps):
+            job.step(warmup + i)
+        e1.record(stream)
+        e1.synchronize()
+        clk.mark(False)
+    torch.cuda.synchronize(dev)
+    job.check_status()
+    return e0.elapsed_time(e1) / steps, clk.summary()
+
+
+SECONDARY = ("decode", "long_context", "many_short")
+
+
+def run_secondary(args, dev, stream, gpu_index):
+    """The other workloads of the benchmark spec, each timed like the headline one: the
+    decode step kernel (B=128 H=8 d_qk=256 d_v=512, state resident in HBM), the
+    long-context layer and the many-short-sequences layer.  One entry each with
+    its own roofline fraction; the headline value stays the 7B-like layer."""
+    hbm, bf16_peak, _, peak_src = peaks()
+    out = []
+    for name in SECONDARY:
+        if name == args.workload:
+            continue
+        w = workload_for_rank(name, 0)
+        inp = make_inputs(w)
+        job = _Decode(w, inp, dev, stream) if w.steps else _Sequence(w, inp, dev, stream)
+        steps = min(args.steps, 100 if w.steps else 50)
+        ms, clocks = time_job(job, steps, args.warmup, stream, dev, gpu_index)
+        bytes_, flops = algorithmic(w)
+        gbs = bytes_ / (ms * 1e-3) / 1e9
+        out.append({"workload": name, "kernel": job.kernel, "ms_per_step": ms,
+                    "value": tokens_per_step(w) / (ms * 1e-3), "unit": UNIT,
+                    "hbm_gbs": gbs, "tflops": flops / (ms * 1e-3) / 1e12,
+                    "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                                 "frac": gbs / hbm, "peak_source": peak_src,
+                                 "algorithmic_bytes_per_launch": bytes_,
+                                 "traffic": traffic_for(kernel_source_sha(), w)},
+                    "gpu_launches": steps * job.launches, "steps": steps, "clocks": clocks,
+                    "config": config_of(w, {"l2": "working set larger than L2 (126 MB)"})})
+        del job, inp
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     from xlstm_mlstm_matrix_b200 import capi, inputs
@@ -553,6 +610,9 @@ def run_ours(args, rank, world, local_rank):
         }
         if world == 1 and not args.no_cpu_baseline:
             line["cpu_baseline"] = cpu_baseline(w, inp, budget_s=args.ref_budget, gated=gated)
+        if world == 1 and not args.no_secondary:
+            gi = local_rank if os.environ.get("CUDA_VISIBLE_DEVICES") is None else 0
+            line["secondary"] = run_secondary(args, dev, stream, gi)
         print(json.dumps(line), flush=True)
 
 
@@ -646,6 +706,8 @@ def main():
     ap.add_argument("--output", choices=["plain", "gated-bf16"], default="plain",
                     help="gated-bf16: the fused output stage (h = sigmoid(o~) h~, bf16 o~ and h)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--no-secondary", action="store_true",
+                    help="skip the decode, long-context and many-short entries of the line")
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")
     ap.add_argument("--H", type=int, default=0, help="override the head count (profiling)")
     ap.add_argument("--T", type=int, default=0, help="override the sequence length (profiling)")

@@ -102,7 +102,12 @@ typedef struct {
  *                      (desc) bytes a long sequence with few heads runs as
  *                      parallel segments.  Calls sharing a workspace must not
  *                      overlap on the device.
- * Chunk lengths: 0 (= 64), 16, 32, 64; others return XLSTM_ERR_UNSUPPORTED.
+ * Chunk lengths: 0 (= 64) and 64 for both input types; 16 and 32 for fp32
+ * inputs only.  Every other length (128 and 256 among them), and 16 or 32 with
+ * bf16 inputs, returns XLSTM_ERR_UNSUPPORTED: the tensor-core kernel that runs
+ * bf16 inputs holds the state, its readout copy and one chunk's accumulators in
+ * tensor memory, which fixes its chunk at 64 tokens.  The chunk length is an
+ * evaluation order, not part of the method: results differ only by rounding.
  * Outputs must not overlap inputs.  T = 0 copies the state through.
  */
 XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise(
@@ -199,9 +204,14 @@ XLSTM_API xlstm_status_t xlstm_mlstm_step(
  *   - All calls share the one array: calls that overlap on the device (other
  *     streams, other host threads) race on it.  Each call clears the part that
  *     must start at zero (the status block) on its stream before its kernel.
- *   - The device status block lives in that array and is not readable through
- *     this API; use xlstm_mlstm_fwd_chunkwise with a workspace when the status
- *     of the device-side waits is needed.
+ *   - The device status block lives at the start of that array; read it after
+ *     the call's stream with xlstm_mlstm_noalloc_status.
+ *   - The array holds only the status block, never segment summaries, so this
+ *     call always runs a sequence in one piece: a long sequence with few heads
+ *     (e.g. 8 heads of 65536 tokens) takes about ten times as long as through
+ *     xlstm_mlstm_fwd_chunkwise given xlstm_mlstm_workspace_size_parallel bytes.
+ *   - The device address is cached per device for the life of the process: do
+ *     not use this call across cudaDeviceReset on a device.
  */
 XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise_noalloc(
     const xlstm_mlstm_desc_t *desc,
@@ -210,6 +220,17 @@ XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise_noalloc(
     const float *C_in, const float *n_in, const float *m_in,
     float *h_out, float *C_out, float *n_out, float *m_out,
     cudaStream_t stream);
+
+/*
+ * The device status block of the last xlstm_mlstm_fwd_chunkwise_noalloc call on
+ * the current device (the allocation-free counterpart of
+ * xlstm_mlstm_workspace_status; the pages have no counterpart either): copies
+ * the block to the host on `stream` and waits for that stream, so call it after
+ * the call you want to check, on its stream.  Returns the block's code (XLSTM_OK
+ * or XLSTM_ERR_TIMEOUT) and, if where != NULL, the code of the wait that gave
+ * up; XLSTM_ERR_CUDA if the copy fails.  Allocates nothing.
+ */
+XLSTM_API xlstm_status_t xlstm_mlstm_noalloc_status(int32_t *where, cudaStream_t stream);
 
 /* Workspace bytes xlstm_mlstm_fwd_chunkwise needs for desc (>= 256), or 0 for
  * a NULL desc. */

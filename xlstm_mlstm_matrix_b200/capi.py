@@ -22,7 +22,7 @@ EXPORTED = ("xlstm_mlstm_fwd_chunkwise", "xlstm_mlstm_fwd_recurrent", "xlstm_mls
             "xlstm_mlstm_workspace_size", "xlstm_mlstm_workspace_status", "xlstm_status_string",
             "xlstm_mlstm_version", "xlstm_mlstm_chunkwise_kernel", "xlstm_mlstm_test_timeout_next",
             "xlstm_mlstm_fwd_chunkwise_noalloc", "xlstm_mlstm_workspace_size_parallel",
-            "xlstm_mlstm_fwd_chunkwise_out")
+            "xlstm_mlstm_fwd_chunkwise_out", "xlstm_mlstm_noalloc_status")
 
 
 class xlstm_mlstm_desc_t(ctypes.Structure):
@@ -70,6 +70,8 @@ def load(path: str = LIB_PATH):
     lib.xlstm_mlstm_workspace_size_parallel.restype = sz
     lib.xlstm_mlstm_workspace_status.argtypes = [vp, ctypes.POINTER(ctypes.c_int32), vp]
     lib.xlstm_mlstm_workspace_status.restype = st
+    lib.xlstm_mlstm_noalloc_status.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
+    lib.xlstm_mlstm_noalloc_status.restype = st
     lib.xlstm_status_string.argtypes = [st]
     lib.xlstm_status_string.restype = ctypes.c_char_p
     lib.xlstm_mlstm_version.argtypes = []
@@ -158,6 +160,13 @@ def xlstm_mlstm_workspace_size_parallel(desc) -> int:
 def xlstm_mlstm_workspace_status(workspace, stream=None):
     where = ctypes.c_int32(0)
     st = load().xlstm_mlstm_workspace_status(_p(workspace), ctypes.byref(where), _s(stream))
+    return int(st), int(where.value)
+
+
+def xlstm_mlstm_noalloc_status(stream=None):
+    """(code, where) of the status block used by the last allocation-free call."""
+    where = ctypes.c_int32(0)
+    st = load().xlstm_mlstm_noalloc_status(ctypes.byref(where), _s(stream))
     return int(st), int(where.value)
 
 

@@ -36,6 +36,15 @@ bool dims_ok(const xlstm_mlstm_desc_t *d) {
 
 size_t elem(const xlstm_mlstm_desc_t *d) { return d->qkv_dtype == XLSTM_BF16 ? 2 : 4; }
 
+// Chunk lengths each path takes: 64 for every input type; 16 and 32 for fp32
+// inputs, which run on the CUDA-core kernel.  bf16 inputs run on the tensor-core
+// kernel, whose tile plan fixes L = 64; other lengths are refused, not rerouted.
+bool chunk_ok(const xlstm_mlstm_desc_t *d) {
+    const int L = d->chunk ? d->chunk : 64;
+    if (L == 64) return true;
+    return d->qkv_dtype == XLSTM_F32 && (L == 16 || L == 32);
+}
+
 // Shared validation of the two sequence calls.
 // h_elem: bytes per element of h; o (optional input, o_elem bytes per element) is
 // the output-gate pre-activation tensor of the chunkwise output stage.
@@ -117,8 +126,7 @@ namespace {
 xlstm_status_t run_chunkwise(const xlstm_mlstm_desc_t *desc, FwdArgs a, xlstm_status_t st, void *workspace,
                              size_t workspace_bytes, cudaStream_t stream) {
     if (st != XLSTM_OK) return st;
-    const int L = desc->chunk ? desc->chunk : 64;
-    if (L != 16 && L != 32 && L != 64) return XLSTM_ERR_UNSUPPORTED;
+    if (!chunk_ok(desc)) return XLSTM_ERR_UNSUPPORTED;
     if (!workspace || workspace_bytes < xlstm_mlstm_workspace_size(desc)) return XLSTM_ERR_WORKSPACE;
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return XLSTM_ERR_INVALID_ARG;
     a.status = static_cast<int32_t *>(workspace);
@@ -250,8 +258,7 @@ const char *xlstm_mlstm_version(void) { return "xlstm_mlstm_b200 0.1 (sm_100a)";
 
 const char *xlstm_mlstm_chunkwise_kernel(const xlstm_mlstm_desc_t *desc) {
     if (!desc || !dims_ok(desc)) return "none";
-    const int L = desc->chunk ? desc->chunk : 64;
-    if (L != 16 && L != 32 && L != 64) return "none";
+    if (!chunk_ok(desc)) return "none";
     FwdArgs a = pack(desc, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
                      nullptr, nullptr, nullptr, nullptr);
     if (a.T == 0) return "copy";

@@ -55,3 +55,10 @@ extern "C" xlstm_status_t xlstm_mlstm_fwd_chunkwise_noalloc(
     return xlstm_mlstm_fwd_chunkwise(desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in, h_out, C_out, n_out,
                                      m_out, scratch, kNoAllocScratchBytes, stream);
 }
+
+extern "C" xlstm_status_t xlstm_mlstm_noalloc_status(int32_t *where, cudaStream_t stream) {
+    void *scratch = nullptr;
+    const xlstm_status_t st = scratch_address(&scratch);
+    if (st != XLSTM_OK) return st;
+    return xlstm_mlstm_workspace_status(scratch, where, stream);
+}
