@@ -232,6 +232,48 @@ XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise_noalloc(
  */
 XLSTM_API xlstm_status_t xlstm_mlstm_noalloc_status(int32_t *where, cudaStream_t stream);
 
+/*
+ * Sequences cut along T (e.g. across GPUs).  Over a stretch of tokens the
+ * recurrence (xLSTM page, "mLSTM (matrix LSTM)" eq. 1-2 with the stabilizer of
+ * the "sLSTM" section) maps the entering state to the leaving one affinely:
+ * the true state is scaled by e^F (F = the stretch's summed f~) and the
+ * stretch's own contribution is added.  A stretch is therefore summarised by F
+ * and by the state it leaves from a zero state whose stabilizer starts at -inf:
+ *   C_seg = sum_t e^{u_t - u*} v_t k_t^T,  n_seg = sum_t e^{u_t - u*} k_t,
+ *   m_seg = F + u*,  with F_t = sum_{r<=t} f~_r, u_t = i~_t - F_t, u* = max_t u_t.
+ *
+ * xlstm_mlstm_segment_summary: the summary of each (b, h) sequence of desc.
+ *   k [B][H][T][d_qk], v [B][H][T][d_v] (desc->qkv_dtype), i_pre, f_pre [B][H][T];
+ *   C_seg [B][H][d_v][d_qk], n_seg [B][H][d_qk] (fp32), F_m [B][H][2] (float64:
+ *   F, m_seg).  Runs on the tcgen05 summary kernel: bf16 inputs, d_qk in
+ *   {64, 128, 256}, d_v a multiple of 64, T a multiple of 64 and at most 65536,
+ *   chunk 0 or 64; other descs return XLSTM_ERR_UNSUPPORTED.  Workspace and
+ *   status block as for xlstm_mlstm_fwd_chunkwise (>= 256 bytes).
+ */
+XLSTM_API xlstm_status_t xlstm_mlstm_segment_summary(
+    const xlstm_mlstm_desc_t *desc, const void *k, const void *v,
+    const float *i_pre, const float *f_pre,
+    float *C_seg, float *n_seg, double *F_m,
+    void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
+ * xlstm_mlstm_combine_states: the state after nsum summarised stretches in order,
+ * chained onto (C_in, n_in, m_in) (all NULL: zero state, m = 0):
+ *   m' = max(F + m, m_seg),  C' = e^{F+m-m'} C + e^{m_seg-m'} C_seg  (n likewise),
+ * every coefficient <= 1, the gauge chain in float64 with each m' rounded to the
+ * fp32 it is stored as.  The result carries the recurrence's canonical m, so it
+ * is the entry state of the next stretch for xlstm_mlstm_fwd_chunkwise.
+ *   C_seg [nsum][B][H][d_v][d_qk], n_seg [nsum][B][H][d_qk], F_m [nsum][B][H][2];
+ *   C_out, n_out, m_out: required, must not overlap the inputs.
+ * desc gives B, H, d_qk, d_v; its T, dtype and chunk are ignored.  nsum = 0
+ * copies the entry state (or writes the zero state).
+ */
+XLSTM_API xlstm_status_t xlstm_mlstm_combine_states(
+    const xlstm_mlstm_desc_t *desc, int32_t nsum,
+    const float *C_in, const float *n_in, const float *m_in,
+    const float *C_seg, const float *n_seg, const double *F_m,
+    float *C_out, float *n_out, float *m_out, cudaStream_t stream);
+
 /* Workspace bytes xlstm_mlstm_fwd_chunkwise needs for desc (>= 256), or 0 for
  * a NULL desc. */
 XLSTM_API size_t xlstm_mlstm_workspace_size(const xlstm_mlstm_desc_t *desc);

@@ -22,7 +22,8 @@ EXPORTED = ("xlstm_mlstm_fwd_chunkwise", "xlstm_mlstm_fwd_recurrent", "xlstm_mls
             "xlstm_mlstm_workspace_size", "xlstm_mlstm_workspace_status", "xlstm_status_string",
             "xlstm_mlstm_version", "xlstm_mlstm_chunkwise_kernel", "xlstm_mlstm_test_timeout_next",
             "xlstm_mlstm_fwd_chunkwise_noalloc", "xlstm_mlstm_workspace_size_parallel",
-            "xlstm_mlstm_fwd_chunkwise_out", "xlstm_mlstm_noalloc_status")
+            "xlstm_mlstm_fwd_chunkwise_out", "xlstm_mlstm_noalloc_status", "xlstm_mlstm_segment_summary",
+            "xlstm_mlstm_combine_states")
 
 
 class xlstm_mlstm_desc_t(ctypes.Structure):
@@ -72,6 +73,10 @@ def load(path: str = LIB_PATH):
     lib.xlstm_mlstm_workspace_status.restype = st
     lib.xlstm_mlstm_noalloc_status.argtypes = [ctypes.POINTER(ctypes.c_int32), vp]
     lib.xlstm_mlstm_noalloc_status.restype = st
+    lib.xlstm_mlstm_segment_summary.argtypes = [dp] + [vp] * 7 + [vp, sz, vp]
+    lib.xlstm_mlstm_segment_summary.restype = st
+    lib.xlstm_mlstm_combine_states.argtypes = [dp, ctypes.c_int32] + [vp] * 9 + [vp]
+    lib.xlstm_mlstm_combine_states.restype = st
     lib.xlstm_status_string.argtypes = [st]
     lib.xlstm_status_string.restype = ctypes.c_char_p
     lib.xlstm_mlstm_version.argtypes = []
@@ -147,6 +152,19 @@ def xlstm_mlstm_step(desc, q, k, v, i_pre, f_pre, C, n, m, h_out, C_new, n_new, 
     return load().xlstm_mlstm_step(ctypes.byref(desc), _p(q), _p(k), _p(v), _p(i_pre), _p(f_pre),
                                    _p(C), _p(n), _p(m), _p(h_out), _p(C_new), _p(n_new),
                                    _p(m_new), _s(stream))
+
+
+def xlstm_mlstm_segment_summary(desc, k, v, i_pre, f_pre, C_seg, n_seg, F_m, workspace, workspace_bytes,
+                                stream=None) -> int:
+    return load().xlstm_mlstm_segment_summary(ctypes.byref(desc), _p(k), _p(v), _p(i_pre), _p(f_pre), _p(C_seg),
+                                               _p(n_seg), _p(F_m), _p(workspace), int(workspace_bytes), _s(stream))
+
+
+def xlstm_mlstm_combine_states(desc, nsum, C_in, n_in, m_in, C_seg, n_seg, F_m, C_out, n_out, m_out,
+                               stream=None) -> int:
+    return load().xlstm_mlstm_combine_states(ctypes.byref(desc), int(nsum), _p(C_in), _p(n_in), _p(m_in),
+                                              _p(C_seg), _p(n_seg), _p(F_m), _p(C_out), _p(n_out), _p(m_out),
+                                              _s(stream))
 
 
 def xlstm_mlstm_workspace_size(desc) -> int:
@@ -280,3 +298,39 @@ def step(q, k, v, i_pre, f_pre, state, qk_scale=None, stream=None, out=None, inp
     check(xlstm_mlstm_step(desc, q, k, v, i_pre, f_pre, C, n, m, h, C1, n1, m1, stream),
           "xlstm_mlstm_step")
     return h, (C1, n1, m1)
+
+
+def summary(k, v, i_pre, f_pre, stream=None, workspace=None):
+    """Summary of each (b, h) stretch through xlstm_mlstm_segment_summary:
+    (C_seg [B,H,dv,dqk] fp32, n_seg [B,H,dqk] fp32, F_m [B,H,2] float64)."""
+    import torch
+    B, H, T, dqk = k.shape
+    dv = v.shape[-1]
+    desc = make_desc(B, H, T, dqk, dv, _dtype_code(k), 1.0, 0)
+    dev = k.device
+    C = torch.empty(B, H, dv, dqk, device=dev, dtype=torch.float32)
+    n = torch.empty(B, H, dqk, device=dev, dtype=torch.float32)
+    Fm = torch.empty(B, H, 2, device=dev, dtype=torch.float64)
+    if workspace is None:
+        workspace = torch.empty(256, device=dev, dtype=torch.uint8)
+    stream = stream if stream is not None else torch.cuda.current_stream(dev)
+    check(xlstm_mlstm_segment_summary(desc, k, v, i_pre, f_pre, C, n, Fm, workspace, workspace.numel(), stream),
+          "xlstm_mlstm_segment_summary")
+    return C, n, Fm
+
+
+def combine(C_seg, n_seg, F_m, state=None, stream=None):
+    """State after the stacked summaries (leading axis = stretch, in order)
+    chained onto state (or the zero state), through xlstm_mlstm_combine_states."""
+    import torch
+    S, B, H, dv, dqk = C_seg.shape
+    desc = make_desc(B, H, 1, dqk, dv, XLSTM_F32, 1.0, 0)
+    dev = C_seg.device
+    C1 = torch.empty(B, H, dv, dqk, device=dev, dtype=torch.float32)
+    n1 = torch.empty(B, H, dqk, device=dev, dtype=torch.float32)
+    m1 = torch.empty(B, H, device=dev, dtype=torch.float32)
+    C0, n0, m0 = state if state is not None else (None, None, None)
+    stream = stream if stream is not None else torch.cuda.current_stream(dev)
+    check(xlstm_mlstm_combine_states(desc, S, C0, n0, m0, C_seg, n_seg, F_m, C1, n1, m1, stream),
+          "xlstm_mlstm_combine_states")
+    return C1, n1, m1

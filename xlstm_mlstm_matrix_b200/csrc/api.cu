@@ -231,6 +231,67 @@ xlstm_status_t xlstm_mlstm_step(const xlstm_mlstm_desc_t *desc, const void *q, c
     return xlstm::launch_step(a, stream) == cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;
 }
 
+xlstm_status_t xlstm_mlstm_segment_summary(const xlstm_mlstm_desc_t *desc, const void *k, const void *v,
+                                           const float *i_pre, const float *f_pre, float *C_seg, float *n_seg,
+                                           double *F_m, void *workspace, size_t workspace_bytes,
+                                           cudaStream_t stream) {
+    if (!desc || !dims_ok(desc) || desc->T < 1) return XLSTM_ERR_INVALID_ARG;
+    const void *req[] = {k, v, i_pre, f_pre, C_seg, n_seg, F_m};
+    for (const void *p : req)
+        if (!p || !aligned16(p)) return XLSTM_ERR_INVALID_ARG;
+    const size_t BH = (size_t)desc->B * desc->H, T = (size_t)desc->T, e = elem(desc);
+    const Range ins[] = {rg(k, BH * T * desc->d_qk * e), rg(v, BH * T * desc->d_v * e), rg(i_pre, BH * T * 4),
+                         rg(f_pre, BH * T * 4)};
+    const Range outs[] = {rg(C_seg, BH * desc->d_v * desc->d_qk * 4), rg(n_seg, BH * desc->d_qk * 4),
+                          rg(F_m, BH * 2 * sizeof(double))};
+    for (const Range &o : outs) {
+        for (const Range &i : ins)
+            if (overlap(o, i)) return XLSTM_ERR_INVALID_ARG;
+        for (const Range &o2 : outs)
+            if (&o2 != &o && overlap(o, o2)) return XLSTM_ERR_INVALID_ARG;
+    }
+    FwdArgs a = pack(desc, nullptr, k, v, i_pre, f_pre, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr,
+                     nullptr);
+    if (!chunk_ok(desc) || !xlstm::summary_supported(a)) return XLSTM_ERR_UNSUPPORTED;
+    if (!workspace || workspace_bytes < kWorkspaceBytes) return XLSTM_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return XLSTM_ERR_INVALID_ARG;
+    a.status = static_cast<int32_t *>(workspace);
+    if (cudaMemsetAsync(workspace, 0, 16, stream) != cudaSuccess) return XLSTM_ERR_CUDA;
+    return xlstm::launch_summary(a, C_seg, n_seg, F_m, stream) == cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;
+}
+
+xlstm_status_t xlstm_mlstm_combine_states(const xlstm_mlstm_desc_t *desc, int32_t nsum, const float *C_in,
+                                          const float *n_in, const float *m_in, const float *C_seg,
+                                          const float *n_seg, const double *F_m, float *C_out, float *n_out,
+                                          float *m_out, cudaStream_t stream) {
+    if (!desc) return XLSTM_ERR_INVALID_ARG;
+    xlstm_mlstm_desc_t d = *desc;
+    d.T = 1;
+    if (!dims_ok(&d) || nsum < 0) return XLSTM_ERR_INVALID_ARG;
+    const int ns = (C_in != nullptr) + (n_in != nullptr) + (m_in != nullptr);
+    if (ns != 0 && ns != 3) return XLSTM_ERR_INVALID_ARG;
+    if (nsum > 0 && (!C_seg || !n_seg || !F_m)) return XLSTM_ERR_INVALID_ARG;
+    if (!C_out || !n_out || !m_out) return XLSTM_ERR_INVALID_ARG;
+    const void *all[] = {C_in, n_in, m_in, C_seg, n_seg, F_m, C_out, n_out, m_out};
+    for (const void *p : all)
+        if (!aligned16(p)) return XLSTM_ERR_INVALID_ARG;
+    const size_t BH = (size_t)d.B * d.H, S = (size_t)nsum;
+    const Range ins[] = {rg(C_in, BH * d.d_v * d.d_qk * 4), rg(n_in, BH * d.d_qk * 4), rg(m_in, BH * 4),
+                         rg(C_seg, S * BH * d.d_v * d.d_qk * 4), rg(n_seg, S * BH * d.d_qk * 4),
+                         rg(F_m, S * BH * 2 * sizeof(double))};
+    const Range outs[] = {rg(C_out, BH * d.d_v * d.d_qk * 4), rg(n_out, BH * d.d_qk * 4), rg(m_out, BH * 4)};
+    for (const Range &o : outs) {
+        for (const Range &i : ins)
+            if (overlap(o, i)) return XLSTM_ERR_INVALID_ARG;
+        for (const Range &o2 : outs)
+            if (&o2 != &o && overlap(o, o2)) return XLSTM_ERR_INVALID_ARG;
+    }
+    return xlstm::launch_combine((int)BH, d.d_v, d.d_qk, nsum, C_in, n_in, m_in, C_seg, n_seg, F_m, C_out, n_out,
+                                 m_out, stream) == cudaSuccess
+               ? XLSTM_OK
+               : XLSTM_ERR_CUDA;
+}
+
 xlstm_status_t xlstm_mlstm_workspace_status(const void *workspace, int32_t *where,
                                             cudaStream_t stream) {
     if (!workspace) return XLSTM_ERR_INVALID_ARG;

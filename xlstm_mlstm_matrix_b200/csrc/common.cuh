@@ -40,6 +40,14 @@ struct SegPlan {
 SegPlan segment_plan(const FwdArgs &a);
 // Summaries of segments 0 .. nseg-2 and the entry states of segments 1 .. nseg-1.
 cudaError_t launch_segment_entry_states(const FwdArgs &a, const SegPlan &sp, cudaStream_t s);
+// Summary of a whole sequence (T a multiple of 64, at most 65536 tokens): the state it
+// leaves from a zero state with the stabilizer at -inf, and (F, m_seg) per (b, h).
+bool summary_supported(const FwdArgs &a);
+cudaError_t launch_summary(const FwdArgs &a, float *C_seg, float *n_seg, double *F_m, cudaStream_t s);
+// The state after nsum summaries [nsum][B*H] chained onto (C0, n0, m0) (null: zero state).
+cudaError_t launch_combine(int BH, int dv, int dqk, int nsum, const float *C0, const float *n0, const float *m0,
+                           const float *segC, const float *segN, const double *segS, float *C1, float *n1, float *m1,
+                           cudaStream_t s);
 
 // Device status block layout (first 16 bytes of the workspace).
 enum : int32_t { kStatusCode = 0, kStatusWhere = 1 };

@@ -349,6 +349,8 @@ struct CombineParams {
     const float *C0, *n0, *m0;   // caller's initial state (null: zero state, m = 0)
     float *segC, *segN, *segM;   // summaries in, entry states of segments 1..nsum out (in place)
     const double *segS;
+    float *C1, *n1, *m1;         // non-null: only the state after the last summary is written, here,
+                                 // and the summaries are left as they are
 };
 
 // Entry states, in place over the summaries: slot g becomes the state entering
@@ -392,11 +394,20 @@ __global__ void __launch_bounds__(kCombineThreads) seg_combine_kernel(const Comb
                 const float a = (float)exp(F[j] + m - mp), b = (float)exp(ms[j] - mp);
                 x = make_float4(fmaf(a, x.x, b * y[j].x), fmaf(a, x.y, b * y[j].y), fmaf(a, x.z, b * y[j].z),
                                 fmaf(a, x.w, b * y[j].w));
-                *slot(g0 + j) = x;
-                if (e4 == 0) p.segM[(size_t)(g0 + j) * p.BH + bh] = (float)mp;
+                if (!p.C1) {
+                    *slot(g0 + j) = x;
+                    if (e4 == 0) p.segM[(size_t)(g0 + j) * p.BH + bh] = (float)mp;
+                }
                 m = mp;
             }
         }
+    }
+    if (p.C1) {
+        if (isC)
+            reinterpret_cast<float4 *>(p.C1 + (size_t)bh * p.dv * p.dqk)[e4] = x;
+        else if (p.n1)
+            reinterpret_cast<float4 *>(p.n1 + (size_t)bh * p.dqk)[e4 - nC4] = x;
+        if (e4 == 0 && p.m1) p.m1[bh] = (float)m;
     }
 }
 
@@ -439,12 +450,57 @@ cudaError_t launch_summaries_dqk(const FwdArgs &a, const SegPlan &sp, cudaStream
     q.BH = BH; q.dv = a.dv; q.dqk = DQK; q.nsum = p.nsum;
     q.C0 = a.C0; q.n0 = a.n0; q.m0 = a.m0;
     q.segC = p.segC; q.segN = p.segN; q.segM = reinterpret_cast<float *>(ws + sp.off_M); q.segS = p.segS;
+    q.C1 = q.n1 = q.m1 = nullptr;
     const int n4 = (a.dv * DQK + DQK) / 4;
     seg_combine_kernel<<<dim3((n4 + kCombineThreads - 1) / kCombineThreads, BH), kCombineThreads, 0, s>>>(q);
     return cudaGetLastError();
 }
 
+template <int DQK>
+cudaError_t launch_summary_whole(const FwdArgs &a, float *C_seg, float *n_seg, double *F_m, cudaStream_t s) {
+    using C = SumCfg<DQK>;
+    const int BH = a.B * a.H;
+    CUtensorMap tk, tv;
+    if (!make_tmap_3d_bf16(&tk, a.k, DQK, a.T, BH, 64, 64) || !make_tmap_3d_bf16(&tv, a.v, a.dv, a.T, BH, 64, 64))
+        return cudaErrorInvalidValue;
+    SumParams p;
+    p.T = a.T; p.dv = a.dv; p.nslices = (a.dv + kDvs - 1) / kDvs; p.nsum = 1;
+    p.seg_chunks = a.T / kL; p.BH = BH; p.ig = a.ig; p.fg = a.fg;
+    p.segC = C_seg; p.segN = n_seg; p.segS = F_m; p.status = a.status;
+    auto kern = seg_summary_kernel<DQK>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e != cudaSuccess) return e;
+    kern<<<BH * p.nslices, kSumThreads, C::SMEM, s>>>(tk, tv, p);
+    return cudaGetLastError();
+}
+
 }  // namespace
+
+bool summary_supported(const FwdArgs &a) {
+    return chunkwise_tc_supported(a) && a.T > 0 && a.T % kL == 0 && a.T / kL <= kMaxSegChunks;
+}
+
+cudaError_t launch_summary(const FwdArgs &a, float *C_seg, float *n_seg, double *F_m, cudaStream_t s) {
+    switch (a.dqk) {
+        case 64: return launch_summary_whole<64>(a, C_seg, n_seg, F_m, s);
+        case 128: return launch_summary_whole<128>(a, C_seg, n_seg, F_m, s);
+        case 256: return launch_summary_whole<256>(a, C_seg, n_seg, F_m, s);
+        default: return cudaErrorInvalidValue;
+    }
+}
+
+cudaError_t launch_combine(int BH, int dv, int dqk, int nsum, const float *C0, const float *n0, const float *m0,
+                           const float *segC, const float *segN, const double *segS, float *C1, float *n1, float *m1,
+                           cudaStream_t s) {
+    CombineParams q;
+    q.BH = BH; q.dv = dv; q.dqk = dqk; q.nsum = nsum;
+    q.C0 = C0; q.n0 = n0; q.m0 = m0;
+    q.segC = const_cast<float *>(segC); q.segN = const_cast<float *>(segN); q.segM = nullptr; q.segS = segS;
+    q.C1 = C1; q.n1 = n1; q.m1 = m1;
+    const int n4 = (dv * dqk + dqk) / 4;
+    seg_combine_kernel<<<dim3((n4 + kCombineThreads - 1) / kCombineThreads, BH), kCombineThreads, 0, s>>>(q);
+    return cudaGetLastError();
+}
 
 SegPlan segment_plan(const FwdArgs &a) {
     SegPlan sp;
