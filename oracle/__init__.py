@@ -11,7 +11,9 @@ compiles that file with gcc and marshals numpy float64 arrays into it.
 
 Every function here is pinned by ``tests/test_oracle_pins.py`` against closed
 forms, a brute-force quadratic form, the unstabilized recurrence and a hand
-case; none of those pins calls back into this module's arithmetic.
+case, and the backward by ``tests/test_oracle_backward.py`` against central
+finite differences of the forward and closed forms; none of those pins calls
+back into this module's arithmetic other than the function it checks.
 """
 from __future__ import annotations
 
@@ -48,6 +50,8 @@ def _declare(lib):
     lib.mlstm_oracle_step.argtypes = [i64, i64, i64, i64, dbl] + [ptr] * 12 + [cint]
     lib.mlstm_oracle_output_gate.restype = cint
     lib.mlstm_oracle_output_gate.argtypes = [i64, ptr, ptr, ptr]
+    lib.mlstm_oracle_backward.restype = cint
+    lib.mlstm_oracle_backward.argtypes = [i64, i64, i64, i64, i64, dbl] + [ptr] * 19 + [cint]
     return lib
 
 
@@ -127,6 +131,30 @@ def step(q, k, v, i_pre, f_pre, C, n, m, qk_scale=1.0, threads: int | None = Non
     if rc != 0:
         raise RuntimeError(f"mlstm_oracle_step failed ({rc})")
     return h, C1, n1, m1
+
+
+def backward(q, k, v, i_pre, f_pre, dh, C0=None, n0=None, m0=None, dC=None, dn=None, qk_scale=1.0,
+             threads: int | None = None, lib=None):
+    """Vector-Jacobian product of ``forward`` (mlstm_oracle.c states what is
+    differentiated).  dh [B,H,T,dv] is the upstream gradient of h~; dC
+    [B,H,dv,dqk] and dn [B,H,dqk] (optional) that of the final stored state.
+    Returns dict(dq, dk, dv, di, df, dC0, dn0, dm0) in float64."""
+    q, k, v, ig, fg, dh = (_f64(x) for x in (q, k, v, i_pre, f_pre, dh))
+    C0, n0, m0, dC, dn = (_f64(x) for x in (C0, n0, m0, dC, dn))
+    B, H, T, dqk = q.shape
+    dv = v.shape[-1]
+    assert dh.shape == (B, H, T, dv)
+    out = dict(dq=np.empty((B, H, T, dqk)), dk=np.empty((B, H, T, dqk)), dv=np.empty((B, H, T, dv)),
+               di=np.empty((B, H, T)), df=np.empty((B, H, T)), dC0=np.empty((B, H, dv, dqk)),
+               dn0=np.empty((B, H, dqk)), dm0=np.empty((B, H)))
+    lib = lib or load_library()
+    rc = lib.mlstm_oracle_backward(B, H, T, dqk, dv, float(qk_scale), _p(q), _p(k), _p(v), _p(ig), _p(fg),
+                                   _p(C0), _p(n0), _p(m0), _p(dh), _p(dC), _p(dn),
+                                   *(_p(out[n]) for n in ("dq", "dk", "dv", "di", "df", "dC0", "dn0", "dm0")),
+                                   int(threads or default_threads()))
+    if rc != 0:
+        raise RuntimeError(f"mlstm_oracle_backward failed ({rc})")
+    return out
 
 
 def output_gate(h_tilde, o_pre, lib=None):
