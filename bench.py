@@ -434,6 +434,53 @@ class _Decode:
         return pairs_in, pairs_out
 
 
+class _Backward:
+    """One xlstm_mlstm_bwd_chunkwise over the whole batch per step: gradients of
+    q, k, v and both gates for a synthetic upstream dh (normal, fp32)."""
+
+    def __init__(self, w, inp, dev, stream):
+        import ctypes
+        import torch
+        from xlstm_mlstm_matrix_b200 import capi
+        seq = _Sequence(w, inp, dev, stream)
+        self.ins = seq.ins
+        g = torch.Generator(device=dev).manual_seed(w.seed + 31)
+        self.dh = torch.randn(w.B, w.H, w.T, w.d_v, device=dev, generator=g)
+        f32 = dict(device=dev, dtype=torch.float32)
+        self.outs = [torch.empty(w.B, w.H, w.T, w.d_qk, **f32), torch.empty(w.B, w.H, w.T, w.d_qk, **f32),
+                     torch.empty(w.B, w.H, w.T, w.d_v, **f32), torch.empty(w.B, w.H, w.T, **f32),
+                     torch.empty(w.B, w.H, w.T, **f32)]
+        self.desc = seq.desc
+        wsb = capi.xlstm_mlstm_bwd_workspace_size(self.desc)
+        self.ws = torch.empty(wsb, device=dev, dtype=torch.uint8)
+        P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+        self.fn = capi.load().xlstm_mlstm_bwd_chunkwise
+        self.argv = (ctypes.byref(self.desc), *(P(t) for t in self.ins), P(self.dh), None, None,
+                     *(P(t) for t in self.outs), None, None, None, P(self.ws), wsb,
+                     ctypes.c_void_p(stream.cuda_stream))
+        self.kernel = "backward (chunk entry states, chunk exit adjoints, chunk gradients; fp32 CUDA cores)"
+        self.launches = 5
+        self.name = "xlstm_mlstm_bwd_chunkwise"
+
+    def step(self, i):
+        st = self.fn(*self.argv)
+        if st != 0:
+            from xlstm_mlstm_matrix_b200 import capi
+            raise capi.XlstmError(st, self.name)
+
+    def check_status(self):
+        pass
+
+
+def algorithmic_backward(w):
+    """Bytes of one backward over B*H*T head-tokens: q, k, v, the gates and dh
+    read; dq, dk, dv, di~, df~ written (fp32); the state's gradient if any."""
+    e = 2 if w.dtype == "bf16" else 4
+    N = w.B * w.H * w.T
+    bytes_ = N * ((2 * w.d_qk + w.d_v) * e + 8 + 4 * w.d_v + 4 * (2 * w.d_qk + w.d_v) + 8)
+    return bytes_
+
+
 def time_job(job, steps, warmup, stream, dev, gpu_index):
     """Warm-up, then `steps` launches bracketed by CUDA events on the launch
     stream with clock samples during the timed region: (ms per step, clocks)."""
@@ -458,7 +505,7 @@ def time_job(job, steps, warmup, stream, dev, gpu_index):
     return e0.elapsed_time(e1) / steps, clk.summary()
 
 
-SECONDARY = ("decode", "long_context", "many_short")
+SECONDARY = ("decode", "long_context", "many_short")   # plus the headline layer's backward
 
 
 def run_secondary(args, dev, stream, gpu_index):
@@ -487,6 +534,24 @@ def run_secondary(args, dev, stream, gpu_index):
                                  "traffic": traffic_for(kernel_source_sha(), w)},
                     "gpu_launches": steps * job.launches, "steps": steps, "clocks": clocks,
                     "config": config_of(w, {"l2": "working set larger than L2 (126 MB)"})})
+        del job, inp
+    # the backward of the headline sequence workload
+    w = workload_for_rank(args.workload, 0, args.B, args.H, args.T)
+    if not w.steps:
+        inp = make_inputs(w)
+        job = _Backward(w, inp, dev, stream)
+        steps = min(args.steps, 10)
+        ms, clocks = time_job(job, steps, args.warmup, stream, dev, gpu_index)
+        bytes_ = algorithmic_backward(w)
+        gbs = bytes_ / (ms * 1e-3) / 1e9
+        out.append({"workload": f"{w.name} backward", "kernel": job.kernel, "ms_per_step": ms,
+                    "value": tokens_per_step(w) / (ms * 1e-3), "unit": UNIT, "hbm_gbs": gbs,
+                    "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                                 "frac": gbs / hbm, "peak_source": peak_src,
+                                 "algorithmic_bytes_per_launch": bytes_, "traffic": None},
+                    "gpu_launches": steps * job.launches, "steps": steps, "clocks": clocks,
+                    "config": config_of(w, {"l2": "working set larger than L2 (126 MB)",
+                                            "upstream": "dh ~ N(0, 1) fp32; no final-state gradient"})})
         del job, inp
     return out
 

@@ -233,6 +233,41 @@ XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise_noalloc(
 XLSTM_API xlstm_status_t xlstm_mlstm_noalloc_status(int32_t *where, cudaStream_t stream);
 
 /*
+ * Backward pass (training; xLSTM page, "mLSTM (matrix LSTM)" eq. 1-3 with the
+ * "sLSTM" stabilizer): the vector-Jacobian product of xlstm_mlstm_fwd_chunkwise.
+ * What is differentiated is the readout with the true states,
+ * h_t = C_t q_t / max(|n_t^T q_t|, 1), f_t = e^{f~_t}, i_t = e^{i~_t}; the stabilizer
+ * only stores those states and is a constant of the derivative (h~ does not
+ * depend on it).
+ *   Inputs: desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in as given to the forward
+ *     call (state all NULL: zero state, m = 0); dh [B][H][T][d_v] the upstream
+ *     gradient of h~ (fp32; h~ itself is recomputed); dC_out [B][H][d_v][d_qk]
+ *     and dn_out [B][H][d_qk] that of the final stored state, for a consumer of the
+ *     true state such as the next call of the recurrence (both NULL: zero).
+ *   Outputs (fp32, whatever the input type): dq, dk [B][H][T][d_qk], dv
+ *     [B][H][T][d_v], di_pre, df_pre [B][H][T]; dC_in, dn_in, dm_in: gradients of
+ *     the initial state (each may be NULL; with no initial state they are the
+ *     gradients at the zero state).
+ *   workspace: >= xlstm_mlstm_bwd_workspace_size(desc) bytes, 256-byte aligned
+ *     (the stored state at every chunk entry and the adjoint at every chunk
+ *     exit: about 2 (T / 64) B H d_v d_qk floats).  Chunk: 0 or 64.
+ * Runs on fp32 CUDA cores: the states at chunk entries (sequential in t, with
+ * h~ recomputed in fp32 for dh . h~), the adjoints at chunk exits (sequential
+ * backwards in t), then every chunk's gradients at once.  Outputs must not
+ * overlap inputs.
+ */
+XLSTM_API size_t xlstm_mlstm_bwd_workspace_size(const xlstm_mlstm_desc_t *desc);
+XLSTM_API xlstm_status_t xlstm_mlstm_bwd_chunkwise(
+    const xlstm_mlstm_desc_t *desc,
+    const void *q, const void *k, const void *v,
+    const float *i_pre, const float *f_pre,
+    const float *C_in, const float *n_in, const float *m_in,
+    const float *dh, const float *dC_out, const float *dn_out,
+    float *dq, float *dk, float *dv, float *di_pre, float *df_pre,
+    float *dC_in, float *dn_in, float *dm_in,
+    void *workspace, size_t workspace_bytes, cudaStream_t stream);
+
+/*
  * Sequences cut along T (e.g. across GPUs).  Over a stretch of tokens the
  * recurrence (xLSTM page, "mLSTM (matrix LSTM)" eq. 1-2 with the stabilizer of
  * the "sLSTM" section) maps the entering state to the leaving one affinely:

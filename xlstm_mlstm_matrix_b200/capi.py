@@ -23,7 +23,7 @@ EXPORTED = ("xlstm_mlstm_fwd_chunkwise", "xlstm_mlstm_fwd_recurrent", "xlstm_mls
             "xlstm_mlstm_version", "xlstm_mlstm_chunkwise_kernel", "xlstm_mlstm_test_timeout_next",
             "xlstm_mlstm_fwd_chunkwise_noalloc", "xlstm_mlstm_workspace_size_parallel",
             "xlstm_mlstm_fwd_chunkwise_out", "xlstm_mlstm_noalloc_status", "xlstm_mlstm_segment_summary",
-            "xlstm_mlstm_combine_states")
+            "xlstm_mlstm_combine_states", "xlstm_mlstm_bwd_chunkwise", "xlstm_mlstm_bwd_workspace_size")
 
 
 class xlstm_mlstm_desc_t(ctypes.Structure):
@@ -77,6 +77,10 @@ def load(path: str = LIB_PATH):
     lib.xlstm_mlstm_segment_summary.restype = st
     lib.xlstm_mlstm_combine_states.argtypes = [dp, ctypes.c_int32] + [vp] * 9 + [vp]
     lib.xlstm_mlstm_combine_states.restype = st
+    lib.xlstm_mlstm_bwd_chunkwise.argtypes = [dp] + [vp] * 19 + [vp, sz, vp]
+    lib.xlstm_mlstm_bwd_chunkwise.restype = st
+    lib.xlstm_mlstm_bwd_workspace_size.argtypes = [dp]
+    lib.xlstm_mlstm_bwd_workspace_size.restype = sz
     lib.xlstm_status_string.argtypes = [st]
     lib.xlstm_status_string.restype = ctypes.c_char_p
     lib.xlstm_mlstm_version.argtypes = []
@@ -165,6 +169,18 @@ def xlstm_mlstm_combine_states(desc, nsum, C_in, n_in, m_in, C_seg, n_seg, F_m, 
     return load().xlstm_mlstm_combine_states(ctypes.byref(desc), int(nsum), _p(C_in), _p(n_in), _p(m_in),
                                               _p(C_seg), _p(n_seg), _p(F_m), _p(C_out), _p(n_out), _p(m_out),
                                               _s(stream))
+
+
+def xlstm_mlstm_bwd_chunkwise(desc, q, k, v, i_pre, f_pre, C_in, n_in, m_in, dh, dC_out, dn_out, dq, dk, dv,
+                              di_pre, df_pre, dC_in, dn_in, dm_in, workspace, workspace_bytes, stream=None) -> int:
+    return load().xlstm_mlstm_bwd_chunkwise(
+        ctypes.byref(desc), *(_p(x) for x in (q, k, v, i_pre, f_pre, C_in, n_in, m_in, dh, dC_out, dn_out,
+                                              dq, dk, dv, di_pre, df_pre, dC_in, dn_in, dm_in, workspace)),
+        int(workspace_bytes), _s(stream))
+
+
+def xlstm_mlstm_bwd_workspace_size(desc) -> int:
+    return int(load().xlstm_mlstm_bwd_workspace_size(ctypes.byref(desc)))
 
 
 def xlstm_mlstm_workspace_size(desc) -> int:
@@ -334,3 +350,28 @@ def combine(C_seg, n_seg, F_m, state=None, stream=None):
     check(xlstm_mlstm_combine_states(desc, S, C0, n0, m0, C_seg, n_seg, F_m, C1, n1, m1, stream),
           "xlstm_mlstm_combine_states")
     return C1, n1, m1
+
+
+def bwd(q, k, v, i_pre, f_pre, dh, state=None, dstate=None, qk_scale=None, stream=None, workspace=None):
+    """Backward through xlstm_mlstm_bwd_chunkwise.  Same inputs as ``fwd`` plus the
+    upstream gradients dh of h~ (and dstate = (dC, dn) of the final state, or
+    None).  Returns dict(dq, dk, dv, di, df, dC0, dn0, dm0), fp32."""
+    import torch
+    B, H, T, dqk = q.shape
+    dv = v.shape[-1]
+    scale = (dqk ** -0.5) if qk_scale is None else float(qk_scale)
+    desc = make_desc(B, H, T, dqk, dv, _dtype_code(q), scale, 0)
+    dev = q.device
+    f32 = dict(device=dev, dtype=torch.float32)
+    g = dict(dq=torch.empty(B, H, T, dqk, **f32), dk=torch.empty(B, H, T, dqk, **f32),
+             dv=torch.empty(B, H, T, dv, **f32), di=torch.empty(B, H, T, **f32), df=torch.empty(B, H, T, **f32),
+             dC0=torch.empty(B, H, dv, dqk, **f32), dn0=torch.empty(B, H, dqk, **f32), dm0=torch.empty(B, H, **f32))
+    C0, n0, m0 = state if state is not None else (None, None, None)
+    dC, dn = dstate if dstate is not None else (None, None)
+    if workspace is None:
+        workspace = torch.empty(max(256, xlstm_mlstm_bwd_workspace_size(desc)), device=dev, dtype=torch.uint8)
+    stream = stream if stream is not None else torch.cuda.current_stream(dev)
+    check(xlstm_mlstm_bwd_chunkwise(desc, q, k, v, i_pre, f_pre, C0, n0, m0, dh, dC, dn, g["dq"], g["dk"],
+                                    g["dv"], g["di"], g["df"], g["dC0"], g["dn0"], g["dm0"], workspace,
+                                    workspace.numel(), stream), "xlstm_mlstm_bwd_chunkwise")
+    return g

@@ -292,6 +292,58 @@ xlstm_status_t xlstm_mlstm_combine_states(const xlstm_mlstm_desc_t *desc, int32_
                : XLSTM_ERR_CUDA;
 }
 
+size_t xlstm_mlstm_bwd_workspace_size(const xlstm_mlstm_desc_t *desc) {
+    if (!desc || !dims_ok(desc)) return 0;
+    return xlstm::backward_workspace_bytes(desc->B * desc->H, desc->T, desc->d_qk, desc->d_v);
+}
+
+xlstm_status_t xlstm_mlstm_bwd_chunkwise(const xlstm_mlstm_desc_t *desc, const void *q, const void *k,
+                                         const void *v, const float *i_pre, const float *f_pre,
+                                         const float *C_in, const float *n_in, const float *m_in,
+                                         const float *dh, const float *dC_out, const float *dn_out, float *dq,
+                                         float *dk, float *dv, float *di_pre, float *df_pre, float *dC_in,
+                                         float *dn_in, float *dm_in, void *workspace, size_t workspace_bytes,
+                                         cudaStream_t stream) {
+    if (!desc || !dims_ok(desc)) return XLSTM_ERR_INVALID_ARG;
+    const int ns = (C_in != nullptr) + (n_in != nullptr) + (m_in != nullptr);
+    if (ns != 0 && ns != 3) return XLSTM_ERR_INVALID_ARG;
+    if ((dC_out == nullptr) != (dn_out == nullptr)) return XLSTM_ERR_INVALID_ARG;
+    if (desc->T > 0 && (!q || !k || !v || !i_pre || !f_pre || !dh || !dq || !dk || !dv || !di_pre || !df_pre))
+        return XLSTM_ERR_INVALID_ARG;
+    const void *all[] = {q, k, v, i_pre, f_pre, C_in, n_in, m_in, dh, dC_out, dn_out,
+                         dq, dk, dv, di_pre, df_pre, dC_in, dn_in, dm_in};
+    for (const void *p : all)
+        if (!aligned16(p)) return XLSTM_ERR_INVALID_ARG;
+    const size_t BH = (size_t)desc->B * desc->H, T = (size_t)desc->T, e = elem(desc);
+    const size_t sC = BH * desc->d_v * desc->d_qk * 4, sn = BH * desc->d_qk * 4, sm = BH * 4;
+    const Range ins[] = {rg(q, BH * T * desc->d_qk * e), rg(k, BH * T * desc->d_qk * e), rg(v, BH * T * desc->d_v * e),
+                         rg(i_pre, BH * T * 4), rg(f_pre, BH * T * 4), rg(C_in, sC), rg(n_in, sn), rg(m_in, sm),
+                         rg(dh, BH * T * desc->d_v * 4), rg(dC_out, sC),
+                         rg(dn_out, sn)};
+    const Range outs[] = {rg(dq, BH * T * desc->d_qk * 4), rg(dk, BH * T * desc->d_qk * 4),
+                          rg(dv, BH * T * desc->d_v * 4), rg(di_pre, BH * T * 4), rg(df_pre, BH * T * 4),
+                          rg(dC_in, sC), rg(dn_in, sn), rg(dm_in, sm)};
+    for (const Range &o : outs) {
+        for (const Range &i : ins)
+            if (overlap(o, i)) return XLSTM_ERR_INVALID_ARG;
+        for (const Range &o2 : outs)
+            if (&o2 != &o && overlap(o, o2)) return XLSTM_ERR_INVALID_ARG;
+    }
+    if (desc->chunk != 0 && desc->chunk != 64) return XLSTM_ERR_UNSUPPORTED;
+    const size_t need = xlstm_mlstm_bwd_workspace_size(desc);
+    if (!workspace || workspace_bytes < need) return XLSTM_ERR_WORKSPACE;
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return XLSTM_ERR_INVALID_ARG;
+    xlstm::BwdArgs a;
+    a.B = desc->B; a.H = desc->H; a.T = desc->T; a.dqk = desc->d_qk; a.dv = desc->d_v;
+    a.dtype = desc->qkv_dtype; a.scale = desc->qk_scale;
+    a.q = q; a.k = k; a.v = v; a.ig = i_pre; a.fg = f_pre; a.C0 = C_in; a.n0 = n_in; a.m0 = m_in;
+    a.dh = dh; a.dCT = dC_out; a.dnT = dn_out;
+    a.dq = dq; a.dk = dk; a.dv_ = dv; a.di = di_pre; a.df = df_pre; a.dC0 = dC_in; a.dn0 = dn_in; a.dm0 = dm_in;
+    a.workspace = workspace;
+    if (cudaMemsetAsync(workspace, 0, 16, stream) != cudaSuccess) return XLSTM_ERR_CUDA;
+    return xlstm::launch_backward(a, stream) == cudaSuccess ? XLSTM_OK : XLSTM_ERR_CUDA;
+}
+
 xlstm_status_t xlstm_mlstm_workspace_status(const void *workspace, int32_t *where,
                                             cudaStream_t stream) {
     if (!workspace) return XLSTM_ERR_INVALID_ARG;

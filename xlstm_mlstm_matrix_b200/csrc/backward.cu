@@ -1,0 +1,690 @@
+// Backward pass of the mLSTM forward (vector-Jacobian product), chunkwise.
+//
+// What is differentiated: the readout of the xLSTM page's "mLSTM (matrix LSTM)"
+// section, eq. 3 with the true states of eq. 1-2 (h_t = C_t q_t / max(|n_t^T q_t|,
+// 1), f_t = e^{f~_t}, i_t = e^{i~_t}); the stabilizer of the "sLSTM" section only
+// stores those states, so the gauge m is a constant of the derivative.  Every
+// quantity is the true one rescaled by e^{m_t}, so no factor exceeds 1.
+//
+// Per (batch, head) the sequence is cut into chunks of L = 64 tokens:
+//  1. states (CUDA cores, per value slice, sequential in t): the stored state at
+//     the entry of every chunk, and per token the stabilizer m_t, s~_t = n~_t . q_t
+//     and the slice's share of dh_t . h~_t;
+//  2. adjoints (CUDA cores, per value slice, sequential backwards in t): the
+//     adjoint of the state at the exit of every chunk,
+//        dC~ <- f'_t (dC~ + (dh_t / den~_t) q_t^T),   dn~ <- f'_t (dn~ + ds~_t q_t),
+//     with ds~_t = -(dh_t . h~_t / den~_t) sign(s~_t) where |s~_t| > e^{-m_t}, else 0;
+//     it ends as the gradient of the initial state;
+//  3. chunk gradients (CUDA cores, every (b, h, chunk) at once): with F_t the
+//     chunk-local cumulative f~, u_s = i~_s - F_s, entry gauge m_0,
+//        W_ts = e^{u_s + F_t - m_t} (s <= t),  a_t = e^{F_t + m_0 - m_t},
+//        z_t = e^{u_t + F_L - m_L},  DN_t = dh_t / den~_t,
+//        M_ts = W_ts (DN_t . v_s + ds~_t),  E_ts = W_ts (q_t . k_s),
+//     dq = scale (diag(a) (DN C~_0 + ds~ n~_0^T) + M K),
+//     dk = M^T Q + diag(z) (V dC~_ex + 1 dn~_ex^T),   di~_t = k_t . dk_t,
+//     dv = E^T DN + diag(z) K dC~_ex^T,
+//     df~_r = sum of the log-weight gradients of every pair the decay from r
+//             belongs to: intra pairs (s < r <= t, M_ts (q_t . k_s)), entry pairs
+//             (t >= r), exit pairs (s < r) and the entry-to-exit pair.
+// The states kernel also forms each value slice's share of dh_t . h~_t from the
+// state it holds (fp32, so the forward's own rounding of h~ does not enter); a
+// small kernel sums the shares, which every value slice of steps 2 and 3 needs.
+#include <math.h>
+
+#include "common.cuh"
+
+namespace xlstm {
+namespace {
+
+constexpr int kL = 64;
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kRpw = 4;                 // rows per warp (sequential kernels)
+constexpr int kRows = kWarps * kRpw;    // value rows per block
+constexpr int kTok = 16;                // tokens staged per barrier
+
+struct BwdLayout {
+    size_t off_C, off_dC, off_n, off_dn, off_m0, off_mt, off_st, off_gt, off_gp, off_dm, bytes;
+};
+
+size_t al256(size_t x) { return (x + 255) & ~size_t(255); }
+
+BwdLayout bwd_layout(int BH, int T, int dqk, int dv) {
+    BwdLayout l;
+    const size_t NC = (size_t)(T + kL - 1) / kL, slices = (size_t)(dv + kRows - 1) / kRows;
+    l.off_C = 256;
+    l.off_dC = al256(l.off_C + NC * BH * (size_t)dv * dqk * 4);
+    l.off_n = al256(l.off_dC + NC * BH * (size_t)dv * dqk * 4);
+    l.off_dn = al256(l.off_n + NC * BH * (size_t)dqk * 4);
+    l.off_m0 = al256(l.off_dn + NC * BH * (size_t)dqk * 4);
+    l.off_mt = al256(l.off_m0 + NC * BH * 8);
+    l.off_st = al256(l.off_mt + (size_t)BH * T * 8);
+    l.off_gt = al256(l.off_st + (size_t)BH * T * 4);
+    l.off_gp = al256(l.off_gt + (size_t)BH * T * 4);
+    l.off_dm = al256(l.off_gp + slices * BH * (size_t)T * 4);
+    l.bytes = al256(l.off_dm + slices * BH * 4);
+    return l;
+}
+
+struct BwdP {
+    int B, H, T, dqk, dv, slices, NC;
+    float scale;
+    const void *q, *k, *v;
+    const float *ig, *fg, *C0, *n0, *m0, *dh, *dCT, *dnT;
+    float *dq, *dk, *dv_, *di, *df, *dC0, *dn0, *dm0;
+    float *wC, *wdC, *wn, *wdn, *wst, *wgt, *wgp, *wdm;
+    double *wm0, *wmt;
+};
+
+// ---- 1. states at chunk entries, m_t and s~_t per token -----------------------------
+// Layout as the recurrent forward: warp w holds rows [w*kRpw, (w+1)*kRpw) of the
+// block's slice in registers, lane l columns l, l+32, ...; each warp keeps n~.
+template <typename Tin, int MAXC>
+__global__ void __launch_bounds__(kThreads) bwd_states_kernel(BwdP p) {
+    extern __shared__ float sm[];
+    const int dqk = p.dqk, dv = p.dv;
+    float *sq = sm;                          // [kTok][dqk] scaled q
+    float *sk = sq + kTok * dqk;             // [kTok][dqk]
+    float *sv = sk + kTok * dqk;             // [kTok][kRows]
+    float *sdh = sv + kTok * kRows;          // [kTok][kRows] dh of the block's rows
+    float *sg = sdh + kTok * kRows;          // [kTok][2] (i~, f~)
+    float *sgw = sg + 2 * kTok;              // [kTok][kWarps] per-warp shares of dh . h~
+    const int bh = blockIdx.x / p.slices, slice = blockIdx.x % p.slices, row0 = slice * kRows;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const Tin *q = static_cast<const Tin *>(p.q) + (size_t)bh * p.T * dqk;
+    const Tin *k = static_cast<const Tin *>(p.k) + (size_t)bh * p.T * dqk;
+    const Tin *v = static_cast<const Tin *>(p.v) + (size_t)bh * p.T * dv;
+    const float *dh = p.dh + (size_t)bh * p.T * dv;
+    const float *ig = p.ig + (size_t)bh * p.T, *fg = p.fg + (size_t)bh * p.T;
+    float C[kRpw][MAXC], n[MAXC];
+    double m = p.m0 ? (double)p.m0[bh] : 0.0;
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+        const int j = lane + 32 * c;
+        n[c] = (p.n0 && j < dqk) ? p.n0[(size_t)bh * dqk + j] : 0.f;
+#pragma unroll
+        for (int r = 0; r < kRpw; ++r) {
+            const int row = row0 + warp * kRpw + r;
+            C[r][c] = (p.C0 && j < dqk && row < dv) ? p.C0[((size_t)bh * dv + row) * dqk + j] : 0.f;
+        }
+    }
+    for (int t0 = 0; t0 < p.T; t0 += kTok) {
+        const int nt = min(kTok, p.T - t0);
+        __syncthreads();
+        for (int e = tid; e < nt * dqk; e += kThreads) {
+            sq[e] = p.scale * to_f32(q[(size_t)t0 * dqk + e]);
+            sk[e] = to_f32(k[(size_t)t0 * dqk + e]);
+        }
+        for (int e = tid; e < nt * kRows; e += kThreads) {
+            const int tt = e / kRows, r = e % kRows;
+            const bool ok = row0 + r < dv;
+            sv[e] = ok ? to_f32(v[(size_t)(t0 + tt) * dv + row0 + r]) : 0.f;
+            sdh[e] = ok ? dh[(size_t)(t0 + tt) * dv + row0 + r] : 0.f;
+        }
+        if (tid < nt) {
+            sg[2 * tid] = ig[t0 + tid];
+            sg[2 * tid + 1] = fg[t0 + tid];
+        }
+        __syncthreads();
+        for (int tt = 0; tt < nt; ++tt) {
+            const int t = t0 + tt;
+            if (t % kL == 0) {   // the stored state entering chunk t / L
+                const size_t ci = (size_t)(t / kL) * (p.B * p.H) + bh;
+#pragma unroll
+                for (int c = 0; c < MAXC; ++c) {
+                    const int j = lane + 32 * c;
+                    if (j >= dqk) continue;
+#pragma unroll
+                    for (int r = 0; r < kRpw; ++r) {
+                        const int row = row0 + warp * kRpw + r;
+                        if (row < dv) p.wC[(ci * dv + row) * dqk + j] = C[r][c];
+                    }
+                    if (slice == 0 && warp == 0) p.wn[ci * dqk + j] = n[c];
+                }
+                if (slice == 0 && tid == 0) p.wm0[ci] = m;
+            }
+            const double it = sg[2 * tt], ft = sg[2 * tt + 1];
+            const double m_new = fmax(ft + m, it);
+            const float fp = expf((float)(ft + m - m_new)), ip = expf((float)(it - m_new));
+            const float *qt = sq + tt * dqk, *kt = sk + tt * dqk;
+            float s = 0.f, num = 0.f;   // n~ . q and this lane's share of sum_r dh_r (C~ q)_r
+#pragma unroll
+            for (int c = 0; c < MAXC; ++c) {
+                const int j = lane + 32 * c;
+                const float kv = (j < dqk) ? kt[j] : 0.f, qv = (j < dqk) ? qt[j] : 0.f;
+                n[c] = fmaf(fp, n[c], ip * kv);
+                s = fmaf(n[c], qv, s);
+                float cq = 0.f;
+#pragma unroll
+                for (int r = 0; r < kRpw; ++r) {
+                    C[r][c] = fmaf(fp, C[r][c], ip * sv[tt * kRows + warp * kRpw + r] * kv);
+                    cq = fmaf(sdh[tt * kRows + warp * kRpw + r], C[r][c], cq);
+                }
+                num = fmaf(cq, qv, num);
+            }
+            s = warp_sum(s);
+            num = warp_sum(num);
+            const float lower = expf((float)(-m_new));
+            const float den = fabsf(s) > lower ? fabsf(s) : lower;
+            if (lane == 0) sgw[tt * kWarps + warp] = num / den;
+            if (slice == 0 && tid == 0) {
+                p.wmt[(size_t)bh * p.T + t] = m_new;
+                p.wst[(size_t)bh * p.T + t] = s;
+            }
+            m = m_new;
+        }
+        __syncthreads();
+        if (tid < nt) {   // this slice's share of dh_t . h~_t
+            float g = 0.f;
+            for (int w = 0; w < kWarps; ++w) g += sgw[tid * kWarps + w];
+            p.wgp[((size_t)slice * (p.B * p.H) + bh) * p.T + t0 + tid] = g;
+        }
+    }
+}
+
+// ---- dh . h~ per token: the value slices' shares summed in order ---------------------------
+__global__ void __launch_bounds__(kThreads) bwd_gsum_kernel(const float *gp, float *g, size_t n, int slices) {
+    const size_t i = (size_t)blockIdx.x * kThreads + threadIdx.x;
+    if (i >= n) return;
+    float s = 0.f;
+    for (int sl = 0; sl < slices; ++sl) s += gp[(size_t)sl * n + i];
+    g[i] = s;
+}
+
+// The readout's derivative factors of token t: den~_t and ds~_t.
+__device__ __forceinline__ void readout_factors(float s, double m, float g, float &den, float &ds) {
+    const float lower = expf((float)(-m));
+    const bool clamp = !(fabsf(s) > lower);
+    den = clamp ? lower : fabsf(s);
+    ds = clamp ? 0.f : -(g / den) * (s > 0.f ? 1.f : -1.f);
+}
+
+// ---- 2. adjoints at chunk exits, backwards in t -----------------------------------------
+template <typename Tin, int MAXC>
+__global__ void __launch_bounds__(kThreads) bwd_adjoint_kernel(BwdP p) {
+    extern __shared__ float sm[];
+    const int dqk = p.dqk, dv = p.dv;
+    float *sq = sm;                          // [kTok][dqk] scaled q
+    float *sdh = sq + kTok * dqk;            // [kTok][kRows] dh_t / den~_t
+    float *ssc = sdh + kTok * kRows;         // [kTok][2] (ds~_t, f'_t)
+    const int bh = blockIdx.x / p.slices, slice = blockIdx.x % p.slices, row0 = slice * kRows;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const Tin *q = static_cast<const Tin *>(p.q) + (size_t)bh * p.T * dqk;
+    const float *fg = p.fg + (size_t)bh * p.T;
+    const double *mt = p.wmt + (size_t)bh * p.T;
+    const float *st = p.wst + (size_t)bh * p.T, *gt = p.wgt + (size_t)bh * p.T;
+    const float *dh = p.dh + (size_t)bh * p.T * dv;
+    float D[kRpw][MAXC], dn[MAXC];
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+        const int j = lane + 32 * c;
+        dn[c] = (p.dnT && j < dqk) ? p.dnT[(size_t)bh * dqk + j] : 0.f;
+#pragma unroll
+        for (int r = 0; r < kRpw; ++r) {
+            const int row = row0 + warp * kRpw + r;
+            D[r][c] = (p.dCT && j < dqk && row < dv) ? p.dCT[((size_t)bh * dv + row) * dqk + j] : 0.f;
+        }
+    }
+    const double m_init = p.m0 ? (double)p.m0[bh] : 0.0;
+    const int nblk = (p.T + kTok - 1) / kTok;
+    for (int b = nblk - 1; b >= 0; --b) {
+        const int t0 = b * kTok, nt = min(kTok, p.T - t0);
+        __syncthreads();
+        for (int e = tid; e < nt * dqk; e += kThreads) sq[e] = p.scale * to_f32(q[(size_t)t0 * dqk + e]);
+        if (tid < nt) {
+            const int t = t0 + tid;
+            float den, ds;
+            readout_factors(st[t], mt[t], gt[t], den, ds);
+            const double mp = t > 0 ? mt[t - 1] : m_init;
+            ssc[2 * tid] = ds;
+            ssc[2 * tid + 1] = expf((float)((double)fg[t] + mp - mt[t]));
+        }
+        // dh / den~ of the block's rows
+        for (int e = tid; e < nt * kRows; e += kThreads) {
+            const int tt = e / kRows, r = e % kRows, t = t0 + tt;
+            float den, ds;
+            readout_factors(st[t], mt[t], gt[t], den, ds);
+            sdh[e] = (row0 + r < dv) ? dh[(size_t)t * dv + row0 + r] / den : 0.f;
+        }
+        __syncthreads();
+        for (int tt = nt - 1; tt >= 0; --tt) {
+            const int t = t0 + tt;
+            if (t == p.T - 1 || (t + 1) % kL == 0) {   // the adjoint at the exit of chunk t / L
+                const size_t ci = (size_t)(t / kL) * (p.B * p.H) + bh;
+#pragma unroll
+                for (int c = 0; c < MAXC; ++c) {
+                    const int j = lane + 32 * c;
+                    if (j >= dqk) continue;
+#pragma unroll
+                    for (int r = 0; r < kRpw; ++r) {
+                        const int row = row0 + warp * kRpw + r;
+                        if (row < dv) p.wdC[(ci * dv + row) * dqk + j] = D[r][c];
+                    }
+                    if (slice == 0 && warp == 0) p.wdn[ci * dqk + j] = dn[c];
+                }
+            }
+            const float ds = ssc[2 * tt], fp = ssc[2 * tt + 1];
+            const float *qt = sq + tt * dqk;
+#pragma unroll
+            for (int c = 0; c < MAXC; ++c) {
+                const int j = lane + 32 * c;
+                const float qv = (j < dqk) ? qt[j] : 0.f;
+                dn[c] = fp * fmaf(ds, qv, dn[c]);
+#pragma unroll
+                for (int r = 0; r < kRpw; ++r) D[r][c] = fp * fmaf(sdh[tt * kRows + warp * kRpw + r], qv, D[r][c]);
+            }
+        }
+    }
+    // the gradient of the initial state, and this slice's share of dm0
+    float part = 0.f;
+#pragma unroll
+    for (int c = 0; c < MAXC; ++c) {
+        const int j = lane + 32 * c;
+        if (j >= dqk) continue;
+#pragma unroll
+        for (int r = 0; r < kRpw; ++r) {
+            const int row = row0 + warp * kRpw + r;
+            if (row >= dv) continue;
+            const size_t e = ((size_t)bh * dv + row) * dqk + j;
+            if (p.dC0) p.dC0[e] = D[r][c];
+            if (p.C0) part = fmaf(D[r][c], p.C0[e], part);
+        }
+        if (slice == 0 && warp == 0) {
+            if (p.dn0) p.dn0[(size_t)bh * dqk + j] = dn[c];
+            if (p.n0) part = fmaf(dn[c], p.n0[(size_t)bh * dqk + j], part);
+        }
+    }
+    part = warp_sum(part);
+    __shared__ float red[kWarps];
+    if (lane == 0) red[warp] = part;
+    __syncthreads();
+    if (tid == 0) {
+        float s = 0.f;
+        for (int w = 0; w < kWarps; ++w) s += red[w];
+        p.wdm[(size_t)slice * (p.B * p.H) + bh] = s;
+    }
+}
+
+__global__ void bwd_dm0_kernel(const float *part, float *dm0, int BH, int slices) {
+    const int bh = blockIdx.x * blockDim.x + threadIdx.x;
+    if (bh >= BH) return;
+    float s = 0.f;
+    for (int i = 0; i < slices; ++i) s += part[(size_t)i * BH + bh];
+    dm0[bh] = s;
+}
+
+// ---- 3. gradients of every chunk, all chunks at once ------------------------------------
+constexpr int kLd = kL + 1;   // padded row of the L x L matrices
+constexpr int kTd = 33;       // padded row of a 32-wide tile
+
+template <typename Tin>
+__device__ __forceinline__ float ld_in(const Tin *p, size_t i) { return to_f32(p[i]); }
+
+template <typename Tin>
+__global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdP p) {
+    extern __shared__ float sm[];
+    float *Mm = sm;                     // [kL][kLd] M_ts
+    float *Em = Mm + kL * kLd;          // [kL][kLd] E_ts
+    float *Gm = Em + kL * kLd;          // [kL][kLd] S, then G_ts
+    float *tA = Gm + kL * kLd;          // [kL][kTd]
+    float *tB = tA + kL * kTd;          // [kL][kTd]
+    float *tC = tB + kL * kTd;          // [32][kTd]
+    float *sa = tC + 32 * kTd, *sz = sa + kL, *sden = sz + kL, *sds = sden + kL;
+    float *sG0 = sds + kL, *sGx = sG0 + kL, *sdi = sGx + kL, *sdfi = sdi + kL, *red = sdfi + kL;
+    double *su = reinterpret_cast<double *>(red + 2 * kWarps);   // [kL] u_s
+    double *sFm = su + kL;                                       // [kL] F_t - m_t
+
+    const int dqk = p.dqk, dv = p.dv, BH = p.B * p.H;
+    const int c = blockIdx.x % p.NC, bh = blockIdx.x / p.NC;
+    const int t0 = c * kL, L = min(kL, p.T - t0);
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const size_t ci = (size_t)c * BH + bh;
+    const Tin *q = static_cast<const Tin *>(p.q) + ((size_t)bh * p.T + t0) * dqk;
+    const Tin *k = static_cast<const Tin *>(p.k) + ((size_t)bh * p.T + t0) * dqk;
+    const Tin *v = static_cast<const Tin *>(p.v) + ((size_t)bh * p.T + t0) * dv;
+    const float *dh = p.dh + ((size_t)bh * p.T + t0) * dv;
+    const float *C0 = p.wC + ci * dv * dqk, *n0 = p.wn + ci * dqk;
+    const float *Dx = p.wdC + ci * dv * dqk, *dnx = p.wdn + ci * dqk;
+
+    // ---- per-token scalars (float64 gate arithmetic, as in the forward)
+    if (warp == 0) {
+        const double m0 = p.wm0[ci];
+        const double *mt = p.wmt + (size_t)bh * p.T + t0;
+        double F = 0.0;
+        // sequential over 32-token halves: lane l holds tokens l and l + 32
+        double fl[2] = {0.0, 0.0}, il[2] = {0.0, 0.0};
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int t = lane + 32 * h2;
+            fl[h2] = t < L ? (double)p.fg[(size_t)bh * p.T + t0 + t] : 0.0;
+            il[h2] = t < L ? (double)p.ig[(size_t)bh * p.T + t0 + t] : 0.0;
+        }
+        double Ft[2];
+        for (int h2 = 0; h2 < 2; ++h2) {
+            double incl = fl[h2];
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const double y = __shfl_up_sync(0xffffffffu, incl, o);
+                if (lane >= o) incl += y;
+            }
+            Ft[h2] = F + incl;
+            F += __shfl_sync(0xffffffffu, incl, 31);
+        }
+        const double FL = __shfl_sync(0xffffffffu, (L - 1) < 32 ? Ft[0] : Ft[1], (L - 1) & 31);
+        const double mL = mt[L - 1];
+        for (int h2 = 0; h2 < 2; ++h2) {
+            const int t = lane + 32 * h2;
+            if (t < L) {
+                const double m = mt[t];
+                const double u = il[h2] - Ft[h2];
+                su[t] = u;
+                sFm[t] = Ft[h2] - m;
+                sa[t] = expf((float)(Ft[h2] + m0 - m));
+                sz[t] = expf((float)(u + FL - mL));
+                float den, ds;
+                readout_factors(p.wst[(size_t)bh * p.T + t0 + t], m, p.wgt[(size_t)bh * p.T + t0 + t], den, ds);
+                sden[t] = den;
+                sds[t] = ds;
+            } else {
+                su[t] = 0.0; sFm[t] = -INFINITY; sa[t] = 0.f; sz[t] = 0.f; sden[t] = 1.f; sds[t] = 0.f;
+            }
+            sG0[t] = 0.f; sGx[t] = 0.f; sdi[t] = 0.f;
+        }
+        if (lane == 0) red[kWarps] = expf((float)(FL + m0 - mL));   // a_L': entry state carried to the exit
+    }
+    __syncthreads();
+
+    const int tr = tid >> 2;          // output row (token) of this thread
+    const int cq = tid & 3;           // its quarter of the columns
+    // ---- S = Q K^T and P = DN V^T (64 x 64)
+    {
+        float accS[16], accP[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) accS[i] = accP[i] = 0.f;
+        for (int j0 = 0; j0 < dqk; j0 += 32) {
+            for (int e = tid; e < kL * 32; e += kThreads) {
+                const int t = e >> 5, jj = e & 31, j = j0 + jj;
+                const bool ok = t < L && j < dqk;
+                tA[t * kTd + jj] = ok ? p.scale * ld_in(q, (size_t)t * dqk + j) : 0.f;
+                tB[t * kTd + jj] = ok ? ld_in(k, (size_t)t * dqk + j) : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int jj = 0; jj < 32; ++jj) {
+                const float a = tA[tr * kTd + jj];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) accS[i] = fmaf(a, tB[(16 * cq + i) * kTd + jj], accS[i]);
+            }
+            __syncthreads();
+        }
+        for (int r0 = 0; r0 < dv; r0 += 32) {
+            for (int e = tid; e < kL * 32; e += kThreads) {
+                const int t = e >> 5, rr = e & 31, r = r0 + rr;
+                const bool ok = t < L && r < dv;
+                tA[t * kTd + rr] = ok ? dh[(size_t)t * dv + r] / sden[t] : 0.f;
+                tB[t * kTd + rr] = ok ? ld_in(v, (size_t)t * dv + r) : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int rr = 0; rr < 32; ++rr) {
+                const float a = tA[tr * kTd + rr];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) accP[i] = fmaf(a, tB[(16 * cq + i) * kTd + rr], accP[i]);
+            }
+            __syncthreads();
+        }
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+            const int s = 16 * cq + i;
+            const float w = (s <= tr && tr < L) ? expf((float)(su[s] + sFm[tr])) : 0.f;
+            const float Mv = w * (accP[i] + sds[tr]);
+            Mm[tr * kLd + s] = Mv;
+            Em[tr * kLd + s] = w * accS[i];
+            Gm[tr * kLd + s] = (s < tr) ? Mv * accS[i] : 0.f;
+        }
+    }
+    __syncthreads();
+    // intra pairs' share of df~_r: sum over t >= r, s < r of G_ts
+    if (tid < kL) {
+        const int r = tid;
+        float acc = 0.f;
+        for (int t = r; t < L; ++t)
+            for (int s = 0; s < r; ++s) acc += Gm[t * kLd + s];
+        sdfi[r] = acc;
+    }
+    // ---- dq = scale (diag(a) (DN C~_0 + ds~ n~_0^T) + M K); G_t0 = a_t q_t . (DN C~_0 + ds~ n~_0)_t
+    for (int j0 = 0; j0 < dqk; j0 += 32) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        for (int r0 = 0; r0 < dv; r0 += 32) {
+            __syncthreads();
+            for (int e = tid; e < kL * 32; e += kThreads) {
+                const int t = e >> 5, rr = e & 31, r = r0 + rr;
+                tA[t * kTd + rr] = (t < L && r < dv) ? dh[(size_t)t * dv + r] / sden[t] : 0.f;
+            }
+            for (int e = tid; e < 32 * 32; e += kThreads) {
+                const int rr = e >> 5, jj = e & 31, r = r0 + rr, j = j0 + jj;
+                tC[rr * kTd + jj] = (r < dv && j < dqk) ? C0[(size_t)r * dqk + j] : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int rr = 0; rr < 32; ++rr) {
+                const float a = tA[tr * kTd + rr];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(a, tC[rr * kTd + 8 * cq + i], acc[i]);
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < kL * 32; e += kThreads) {
+            const int t = e >> 5, jj = e & 31, j = j0 + jj;
+            const bool ok = t < L && j < dqk;
+            tA[t * kTd + jj] = ok ? p.scale * ld_in(q, (size_t)t * dqk + j) : 0.f;
+            tB[t * kTd + jj] = ok ? ld_in(k, (size_t)t * dqk + j) : 0.f;
+        }
+        __syncthreads();
+        float g0 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int jj = 8 * cq + i, j = j0 + jj;
+            const float A1 = acc[i] + (j < dqk ? sds[tr] * n0[j] : 0.f);
+            float intra = 0.f;
+            for (int s = 0; s <= tr && s < L; ++s) intra = fmaf(Mm[tr * kLd + s], tB[s * kTd + jj], intra);
+            if (tr < L && j < dqk) p.dq[((size_t)bh * p.T + t0 + tr) * dqk + j] = p.scale * (sa[tr] * A1 + intra);
+            g0 = fmaf(tA[tr * kTd + jj], sa[tr] * A1, g0);
+        }
+        g0 += __shfl_xor_sync(0xffffffffu, g0, 1);
+        g0 += __shfl_xor_sync(0xffffffffu, g0, 2);
+        if (cq == 0) sG0[tr] += g0;
+    }
+    // ---- dk = M^T Q + diag(z) (V dC~_ex + 1 dn~_ex^T); di~ = k . dk; G_s,ex = k_s . (exit part)
+    for (int j0 = 0; j0 < dqk; j0 += 32) {
+        float acc[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+        for (int r0 = 0; r0 < dv; r0 += 32) {
+            __syncthreads();
+            for (int e = tid; e < kL * 32; e += kThreads) {
+                const int t = e >> 5, rr = e & 31, r = r0 + rr;
+                tA[t * kTd + rr] = (t < L && r < dv) ? ld_in(v, (size_t)t * dv + r) : 0.f;
+            }
+            for (int e = tid; e < 32 * 32; e += kThreads) {
+                const int rr = e >> 5, jj = e & 31, r = r0 + rr, j = j0 + jj;
+                tC[rr * kTd + jj] = (r < dv && j < dqk) ? Dx[(size_t)r * dqk + j] : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int rr = 0; rr < 32; ++rr) {
+                const float a = tA[tr * kTd + rr];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) acc[i] = fmaf(a, tC[rr * kTd + 8 * cq + i], acc[i]);
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < kL * 32; e += kThreads) {
+            const int t = e >> 5, jj = e & 31, j = j0 + jj;
+            const bool ok = t < L && j < dqk;
+            tA[t * kTd + jj] = ok ? p.scale * ld_in(q, (size_t)t * dqk + j) : 0.f;
+            tB[t * kTd + jj] = ok ? ld_in(k, (size_t)t * dqk + j) : 0.f;
+        }
+        __syncthreads();
+        float di = 0.f, gx = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int jj = 8 * cq + i, j = j0 + jj;
+            const float ex = sz[tr] * (acc[i] + (j < dqk ? dnx[j] : 0.f));
+            float intra = 0.f;
+            for (int s = tr; s < L; ++s) intra = fmaf(Mm[s * kLd + tr], tA[s * kTd + jj], intra);
+            const float dkv = intra + ex;
+            if (tr < L && j < dqk) p.dk[((size_t)bh * p.T + t0 + tr) * dqk + j] = dkv;
+            const float kv = tB[tr * kTd + jj];
+            di = fmaf(kv, dkv, di);
+            gx = fmaf(kv, ex, gx);
+        }
+        di += __shfl_xor_sync(0xffffffffu, di, 1);
+        di += __shfl_xor_sync(0xffffffffu, di, 2);
+        gx += __shfl_xor_sync(0xffffffffu, gx, 1);
+        gx += __shfl_xor_sync(0xffffffffu, gx, 2);
+        if (cq == 0) {
+            sdi[tr] += di;
+            sGx[tr] += gx;
+        }
+    }
+    // ---- dv = E^T DN + diag(z) K dC~_ex^T
+    for (int r0 = 0; r0 < dv; r0 += 32) {
+        float acc[8], ex[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) acc[i] = ex[i] = 0.f;
+        for (int j0 = 0; j0 < dqk; j0 += 32) {
+            __syncthreads();
+            for (int e = tid; e < kL * 32; e += kThreads) {
+                const int t = e >> 5, jj = e & 31, j = j0 + jj;
+                tB[t * kTd + jj] = (t < L && j < dqk) ? ld_in(k, (size_t)t * dqk + j) : 0.f;
+            }
+            for (int e = tid; e < 32 * 32; e += kThreads) {
+                const int rr = e >> 5, jj = e & 31, r = r0 + rr, j = j0 + jj;
+                tC[rr * kTd + jj] = (r < dv && j < dqk) ? Dx[(size_t)r * dqk + j] : 0.f;
+            }
+            __syncthreads();
+#pragma unroll 4
+            for (int jj = 0; jj < 32; ++jj) {
+                const float a = tB[tr * kTd + jj];
+#pragma unroll
+                for (int i = 0; i < 8; ++i) ex[i] = fmaf(a, tC[(8 * cq + i) * kTd + jj], ex[i]);
+            }
+        }
+        __syncthreads();
+        for (int e = tid; e < kL * 32; e += kThreads) {
+            const int t = e >> 5, rr = e & 31, r = r0 + rr;
+            tA[t * kTd + rr] = (t < L && r < dv) ? dh[(size_t)t * dv + r] / sden[t] : 0.f;
+        }
+        __syncthreads();
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const int rr = 8 * cq + i, r = r0 + rr;
+            float intra = 0.f;
+            for (int s = tr; s < L; ++s) intra = fmaf(Em[s * kLd + tr], tA[s * kTd + rr], intra);
+            if (tr < L && r < dv) p.dv_[((size_t)bh * p.T + t0 + tr) * dv + r] = intra + sz[tr] * ex[i];
+        }
+    }
+    // ---- the entry state carried to the exit: G_0,ex = a_L' (<dC~_ex, C~_0> + <dn~_ex, n~_0>)
+    {
+        float part = 0.f;
+        for (size_t e = tid; e < (size_t)dv * dqk; e += kThreads) part = fmaf(Dx[e], C0[e], part);
+        for (int j = tid; j < dqk; j += kThreads) part = fmaf(dnx[j], n0[j], part);
+        part = warp_sum(part);
+        __syncthreads();
+        if (lane == 0) red[warp] = part;
+        __syncthreads();
+        if (tid == 0) {
+            float s = 0.f;
+            for (int w = 0; w < kWarps; ++w) s += red[w];
+            red[kWarps + 1] = red[kWarps] * s;
+        }
+        __syncthreads();
+    }
+    // ---- df~_r and di~_r
+    if (tid < L) {
+        const int r = tid;
+        float acc = sdfi[r] + red[kWarps + 1];
+        for (int t = r; t < L; ++t) acc += sG0[t];
+        for (int s = 0; s < r; ++s) acc += sGx[s];
+        p.df[(size_t)bh * p.T + t0 + r] = acc;
+        p.di[(size_t)bh * p.T + t0 + r] = sdi[r];
+    }
+}
+
+size_t chunk_smem_bytes() {
+    return (size_t)(3 * kL * kLd + 2 * kL * kTd + 32 * kTd + 9 * kL + 2 * kWarps) * sizeof(float) +
+           2 * kL * sizeof(double) + 16;
+}
+
+template <typename Tin>
+cudaError_t launch_bwd_typed(BwdP p, cudaStream_t s) {
+    const int maxc = (p.dqk + 31) / 32;
+    const size_t smem_seq = (size_t)(2 * kTok * p.dqk + 2 * kTok * kRows + 2 * kTok + kTok * kWarps) * sizeof(float);
+    const dim3 gseq(p.B * p.H * p.slices);
+    cudaError_t e;
+#define XLSTM_BWD_SEQ(MC)                                                                              \
+    if (maxc <= MC) {                                                                                  \
+        auto k1 = bwd_states_kernel<Tin, MC>;                                                          \
+        auto k2 = bwd_adjoint_kernel<Tin, MC>;                                                         \
+        if ((e = cudaFuncSetAttribute(k1, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_seq)) \
+            != cudaSuccess) return e;                                                                  \
+        if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem_seq)) \
+            != cudaSuccess) return e;                                                                  \
+        if (p.T > 0) {                                                                                 \
+            k1<<<gseq, kThreads, smem_seq, s>>>(p);                                                    \
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;                                     \
+            const size_t rows = (size_t)p.B * p.H * p.T;                                               \
+            bwd_gsum_kernel<<<(unsigned)((rows + kThreads - 1) / kThreads), kThreads, 0, s>>>(p.wgp, p.wgt, rows, p.slices); \
+            if ((e = cudaGetLastError()) != cudaSuccess) return e;                                     \
+        }                                                                                              \
+        k2<<<gseq, kThreads, smem_seq, s>>>(p);                                                        \
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;                                         \
+    } else
+    XLSTM_BWD_SEQ(1) XLSTM_BWD_SEQ(2) XLSTM_BWD_SEQ(4) XLSTM_BWD_SEQ(8) XLSTM_BWD_SEQ(16) return cudaErrorInvalidValue;
+#undef XLSTM_BWD_SEQ
+    if (p.dm0) {
+        const int BH = p.B * p.H;
+        bwd_dm0_kernel<<<(BH + 255) / 256, 256, 0, s>>>(p.wdm, p.dm0, BH, p.slices);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    if (p.NC == 0) return cudaSuccess;
+    const size_t smem3 = chunk_smem_bytes();
+    auto k3 = bwd_chunk_kernel<Tin>;
+    if ((e = cudaFuncSetAttribute(k3, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem3)) != cudaSuccess)
+        return e;
+    k3<<<p.B * p.H * p.NC, kThreads, smem3, s>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t backward_workspace_bytes(int BH, int T, int dqk, int dv) { return bwd_layout(BH, T, dqk, dv).bytes; }
+
+cudaError_t launch_backward(const BwdArgs &a, cudaStream_t s) {
+    const int BH = a.B * a.H;
+    const BwdLayout l = bwd_layout(BH, a.T, a.dqk, a.dv);
+    char *ws = static_cast<char *>(a.workspace);
+    BwdP p;
+    p.B = a.B; p.H = a.H; p.T = a.T; p.dqk = a.dqk; p.dv = a.dv;
+    p.slices = (a.dv + kRows - 1) / kRows;
+    p.NC = (a.T + kL - 1) / kL;
+    p.scale = a.scale;
+    p.q = a.q; p.k = a.k; p.v = a.v; p.ig = a.ig; p.fg = a.fg;
+    p.C0 = a.C0; p.n0 = a.n0; p.m0 = a.m0; p.dh = a.dh; p.dCT = a.dCT; p.dnT = a.dnT;
+    p.dq = a.dq; p.dk = a.dk; p.dv_ = a.dv_; p.di = a.di; p.df = a.df; p.dC0 = a.dC0; p.dn0 = a.dn0; p.dm0 = a.dm0;
+    p.wC = reinterpret_cast<float *>(ws + l.off_C);
+    p.wdC = reinterpret_cast<float *>(ws + l.off_dC);
+    p.wn = reinterpret_cast<float *>(ws + l.off_n);
+    p.wdn = reinterpret_cast<float *>(ws + l.off_dn);
+    p.wm0 = reinterpret_cast<double *>(ws + l.off_m0);
+    p.wmt = reinterpret_cast<double *>(ws + l.off_mt);
+    p.wst = reinterpret_cast<float *>(ws + l.off_st);
+    p.wgt = reinterpret_cast<float *>(ws + l.off_gt);
+    p.wgp = reinterpret_cast<float *>(ws + l.off_gp);
+    p.wdm = reinterpret_cast<float *>(ws + l.off_dm);
+    return a.dtype == XLSTM_BF16 ? launch_bwd_typed<__nv_bfloat16>(p, s) : launch_bwd_typed<float>(p, s);
+}
+
+}  // namespace xlstm

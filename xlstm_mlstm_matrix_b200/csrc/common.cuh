@@ -49,6 +49,20 @@ cudaError_t launch_combine(int BH, int dv, int dqk, int nsum, const float *C0, c
                            const float *segC, const float *segN, const double *segS, float *C1, float *n1, float *m1,
                            cudaStream_t s);
 
+// Everything one backward launch needs (validated by the C ABI layer).
+struct BwdArgs {
+    int B, H, T, dqk, dv, dtype;
+    float scale;
+    const void *q, *k, *v;
+    const float *ig, *fg, *C0, *n0, *m0;   // forward inputs (null state: zero, m = 0)
+    const float *dh, *dCT, *dnT;           // upstream gradients (dCT, dnT may be null)
+    float *dq, *dk, *dv_, *di, *df;        // gradients of the inputs (fp32)
+    float *dC0, *dn0, *dm0;                // gradients of the initial state (each may be null)
+    void *workspace;                       // backward_workspace_bytes(...)
+};
+size_t backward_workspace_bytes(int BH, int T, int dqk, int dv);
+cudaError_t launch_backward(const BwdArgs &a, cudaStream_t s);
+
 // Device status block layout (first 16 bytes of the workspace).
 enum : int32_t { kStatusCode = 0, kStatusWhere = 1 };
 
