@@ -148,11 +148,12 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def traffic_for(kernel_src_sha: str, workload, gated=False):
+def traffic_for(kernel_src_sha: str, workload, gated=False, chunk=64):
     """DRAM bytes per launch from the committed ncu summary, if it was taken on
     the current kernel source for this workload at its full size (no --B/--H/--T
-    override) and on the plain output path; else None.  workload: a Workload or
-    a workload name (taken at full size)."""
+    override), on the plain output path and at the chunk length it names (64
+    when it names none); else None.  workload: a Workload or a workload name
+    (taken at full size)."""
     from xlstm_mlstm_matrix_b200 import inputs
     name = workload if isinstance(workload, str) else workload.name
     if not isinstance(workload, str) and workload != inputs.WORKLOADS.get(name, None).replace(seed=workload.seed):
@@ -162,7 +163,7 @@ def traffic_for(kernel_src_sha: str, workload, gated=False):
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
-    d = json.load(open(path)).get(name)
+    d = json.load(open(path)).get(name if chunk in (0, 64) else f"{name} L={chunk}")
     if not d or d.get("source_sha") != kernel_src_sha:
         return None
     return d.get("traffic_bytes_per_launch")
@@ -315,10 +316,10 @@ class _Sequence:
     """One chunkwise forward over the whole batch per step (gated: through the
     output stage, bf16 o~ in and bf16 h out)."""
 
-    def __init__(self, w, inp, dev, stream, gated=False):
+    def __init__(self, w, inp, dev, stream, gated=False, chunk=64):
         import torch
         from xlstm_mlstm_matrix_b200 import capi
-        self.w, self.inp = w, inp
+        self.w, self.inp, self.chunk = w, inp, chunk
         bf = w.dtype == "bf16"
         dev_t = lambda x, b: None if x is None else (
             torch.from_numpy(x).to(dev).to(torch.bfloat16) if b else torch.from_numpy(x).to(dev))
@@ -333,7 +334,7 @@ class _Sequence:
                      torch.empty(w.B, w.H, w.d_v, w.d_qk, device=dev),
                      torch.empty(w.B, w.H, w.d_qk, device=dev), torch.empty(w.B, w.H, device=dev)]
         self.desc = capi.make_desc(w.B, w.H, w.T, w.d_qk, w.d_v,
-                                   capi.XLSTM_BF16 if bf else capi.XLSTM_F32, inp["qk_scale"], 64)
+                                   capi.XLSTM_BF16 if bf else capi.XLSTM_F32, inp["qk_scale"], chunk)
         # a workspace large enough for the segment-parallel path: a long sequence with few
         # heads then runs as segment summaries, their combination and the chunkwise kernel
         wsb = capi.xlstm_mlstm_workspace_size_parallel(self.desc)
@@ -509,7 +510,8 @@ def time_job(job, steps, warmup, stream, dev, gpu_index):
     return e0.elapsed_time(e1) / steps, clk.summary()
 
 
-SECONDARY = ("decode", "long_context", "many_short")   # plus the headline layer's backward
+# (workload, chunk length); plus the headline layer's backward
+SECONDARY = (("decode", 0), ("long_context", 64), ("long_context", 128), ("many_short", 64), ("many_short", 128))
 
 
 def run_secondary(args, dev, stream, gpu_index):
@@ -519,26 +521,32 @@ def run_secondary(args, dev, stream, gpu_index):
     its own roofline fraction; the headline value stays the 7B-like layer."""
     hbm, bf16_peak, _, peak_src = peaks()
     out = []
-    for name in SECONDARY:
-        if name == args.workload:
+    inp_of = {}
+    for name, chunk in SECONDARY:
+        if name == args.workload and chunk in (0, args.chunk):
             continue
         w = workload_for_rank(name, 0)
-        inp = make_inputs(w)
-        job = _Decode(w, inp, dev, stream) if w.steps else _Sequence(w, inp, dev, stream)
+        if name not in inp_of:
+            inp_of.clear()
+            inp_of[name] = make_inputs(w)
+        inp = inp_of[name]
+        job = _Decode(w, inp, dev, stream) if w.steps else _Sequence(w, inp, dev, stream, chunk=chunk)
         steps = min(args.steps, 100 if w.steps else 50)
         ms, clocks = time_job(job, steps, args.warmup, stream, dev, gpu_index)
         bytes_, flops = algorithmic(w)
         gbs = bytes_ / (ms * 1e-3) / 1e9
-        out.append({"workload": name, "kernel": job.kernel, "ms_per_step": ms,
+        out.append({"workload": f"{name} L={chunk}" if chunk else name, "kernel": job.kernel, "ms_per_step": ms,
                     "value": tokens_per_step(w) / (ms * 1e-3), "unit": UNIT,
                     "hbm_gbs": gbs, "tflops": flops / (ms * 1e-3) / 1e12,
                     "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
                                  "frac": gbs / hbm, "peak_source": peak_src,
                                  "algorithmic_bytes_per_launch": bytes_,
-                                 "traffic": traffic_for(kernel_source_sha(), w)},
+                                 "traffic": traffic_for(kernel_source_sha(), w, chunk=chunk)},
                     "gpu_launches": steps * job.launches, "steps": steps, "clocks": clocks,
-                    "config": config_of(w, {"l2": "working set larger than L2 (126 MB)"})})
+                    "config": config_of(w, {"l2": "working set larger than L2 (126 MB)",
+                                            **({"chunk": chunk} if chunk else {})})})
         del job, inp
+    inp_of.clear()
     # the backward of the headline sequence workload
     w = workload_for_rank(args.workload, 0, args.B, args.H, args.T)
     if not w.steps:
@@ -573,7 +581,7 @@ def run_ours(args, rank, world, local_rank):
     gated = args.output == "gated-bf16"
     if gated and w.steps:
         raise SystemExit("--output gated-bf16 applies to the sequence workloads")
-    job = _Decode(w, inp, dev, stream) if w.steps else _Sequence(w, inp, dev, stream, gated=gated)
+    job = _Decode(w, inp, dev, stream) if w.steps else _Sequence(w, inp, dev, stream, gated=gated, chunk=args.chunk)
 
     dist = None
     if world > 1:
@@ -657,7 +665,7 @@ def run_ours(args, rank, world, local_rank):
                             if gated else "bf16 q/k/v, fp32 gates; fp32 h and state"), "l2": l2,
                  "parallelism": f"replicas x{world} (independent heads)"}
         if not w.steps:
-            extra["chunk"] = 64
+            extra["chunk"] = args.chunk
         if gated:
             extra["output"] = "gated-bf16"
         line = {
@@ -668,7 +676,7 @@ def run_ours(args, rank, world, local_rank):
             "tflops": world * flops / (ms * 1e-3) / 1e12,
             "hbm_gbs": achieved_gbs,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": hbm, "unit": "GB/s",
-                         "frac": achieved_gbs / hbm, "traffic": traffic_for(src_sha, w, gated),
+                         "frac": achieved_gbs / hbm, "traffic": traffic_for(src_sha, w, gated, args.chunk),
                          "peak_source": peak_src, "kernel": job.kernel,
                          "algorithmic_bytes_per_launch": bytes_, "flops_per_launch": flops,
                          "tensor_frac": flops / (ms * 1e-3) / 1e12 / bf16_peak},
@@ -775,6 +783,8 @@ def main():
     ap.add_argument("--output", choices=["plain", "gated-bf16"], default="plain",
                     help="gated-bf16: the fused output stage (h = sigmoid(o~) h~, bf16 o~ and h)")
     ap.add_argument("--no-e2e", action="store_true", help="skip the host-buffer end-to-end leg")
+    ap.add_argument("--chunk", type=int, choices=[64, 128], default=64,
+                    help="chunk length of the headline sequence workload (128: d_qk <= 128 only)")
     ap.add_argument("--no-secondary", action="store_true",
                     help="skip the decode, long-context and many-short entries of the line")
     ap.add_argument("--B", type=int, default=0, help="override the batch size (profiling)")

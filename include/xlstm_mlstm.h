@@ -103,11 +103,14 @@ typedef struct {
  *                      parallel segments.  Calls sharing a workspace must not
  *                      overlap on the device.
  * Chunk lengths: 0 (= 64) and 64 for both input types; 16 and 32 for fp32
- * inputs only.  Every other length (128 and 256 among them), and 16 or 32 with
- * bf16 inputs, returns XLSTM_ERR_UNSUPPORTED: the tensor-core kernel that runs
- * bf16 inputs holds the state, its readout copy and one chunk's accumulators in
- * tensor memory, which fixes its chunk at 64 tokens.  The chunk length is an
- * evaluation order, not part of the method: results differ only by rounding.
+ * inputs only; 128 for bf16 inputs with d_qk = 64 or 128 and d_v a multiple
+ * of 64 (the shapes the tensor-core kernel takes).  Every other length (256
+ * among them), 16 or 32 with bf16 inputs, and 128 at d_qk = 256 return
+ * XLSTM_ERR_UNSUPPORTED: the tensor-core kernel that runs bf16 inputs holds
+ * the state, its readout copy and one chunk's S and H accumulators in tensor
+ * memory (512 columns), which at d_qk = 256 fits a chunk of 64 tokens only, and
+ * at L = 256 no d_qk.  The chunk length is an evaluation order, not part of the
+ * method: results differ only by rounding.
  * Outputs must not overlap inputs.  T = 0 copies the state through.
  */
 XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise(

@@ -126,14 +126,18 @@ def test_workspace_and_chunk_rules(lib):
     assert call(d, wsb=8) == capi.XLSTM_ERR_WORKSPACE
     d.chunk = 48
     assert call(d) == capi.XLSTM_ERR_UNSUPPORTED
-    # bf16 inputs run on the tensor-core kernel, whose chunk is 64: other lengths are
-    # refused (before any device call), never sent to another kernel
-    for L in (16, 32, 128, 256):
-        d = capi.make_desc(1, 1, 4, 64, 64, capi.XLSTM_BF16, 1.0, L)
-        assert call(d) == capi.XLSTM_ERR_UNSUPPORTED, L
-        assert capi.xlstm_mlstm_chunkwise_kernel(d) == "none", L
-    for L in (0, 64):   # "tcgen05" on a GPU (the driver's tensor-map encoder); not "none" anywhere
-        assert capi.xlstm_mlstm_chunkwise_kernel(capi.make_desc(1, 1, 4, 64, 64, capi.XLSTM_BF16, 1.0, L)) != "none"
+    # bf16 inputs run on the tensor-core kernel, whose chunk is 64, or 128 at d_qk <= 128:
+    # other lengths are refused (before any device call), never sent to another kernel
+    for dqk, L in ((64, 16), (64, 32), (64, 256), (128, 256), (256, 128), (256, 32)):
+        d = capi.make_desc(1, 1, 4, dqk, 64, capi.XLSTM_BF16, 1.0, L)
+        assert call(d) == capi.XLSTM_ERR_UNSUPPORTED, (dqk, L)
+        assert capi.xlstm_mlstm_chunkwise_kernel(d) == "none", (dqk, L)
+    # L = 128 needs a shape the tensor-core kernel takes (d_v a multiple of 64)
+    assert capi.xlstm_mlstm_chunkwise_kernel(capi.make_desc(1, 1, 4, 64, 32, capi.XLSTM_BF16, 1.0, 128)) == "none"
+    for dqk, L in ((64, 0), (64, 64), (256, 64), (64, 128), (128, 128)):
+        # "tcgen05" on a GPU (the driver's tensor-map encoder); not "none" anywhere
+        d = capi.make_desc(1, 1, 4, dqk, 64, capi.XLSTM_BF16, 1.0, L)
+        assert capi.xlstm_mlstm_chunkwise_kernel(d) != "none", (dqk, L)
     # fp32 inputs: the CUDA-core kernel takes 16, 32 and 64
     for L in (16, 32, 64):
         assert capi.xlstm_mlstm_chunkwise_kernel(capi.make_desc(1, 1, 4, 64, 64, capi.XLSTM_F32, 1.0, L)) == "simt"

@@ -33,6 +33,8 @@ struct FwdArgs {
 
 // How a long sequence is cut into segments that run in parallel (nseg = 1: not
 // cut), and where the segment summaries sit in the scratch (byte offsets).
+// seg_chunks counts chunks of kSegChunk tokens, a multiple of the call's chunk length.
+constexpr int kSegChunk = 64;
 struct SegPlan {
     int nseg = 1, seg_chunks = 0;
     size_t off_S = 0, off_M = 0, off_N = 0, off_C = 0, bytes = 0;

@@ -39,6 +39,7 @@ constexpr int kL = 64;            // chunk length (tokens)
 constexpr int kDvs = 128;         // value rows per block
 constexpr int kSumThreads = 256;
 constexpr int kRing = 4;          // weight-ring slots (even: each slot has one producer warp)
+static_assert(kSegChunk == 64, "segment plan in 64-token chunks");
 constexpr int kMinSegChunks = 8;  // shortest segment worth a summary
 constexpr int kMaxSegChunks = 1024;   // longest segment (its per-chunk F offsets sit in shared memory)
 constexpr int kCombineThreads = 256;
@@ -477,7 +478,9 @@ cudaError_t launch_summary_whole(const FwdArgs &a, float *C_seg, float *n_seg, d
 }  // namespace
 
 bool summary_supported(const FwdArgs &a) {
-    return chunkwise_tc_supported(a) && a.T > 0 && a.T % kL == 0 && a.T / kL <= kMaxSegChunks;
+    FwdArgs b = a;
+    b.chunk = kL;   // a summary does not depend on the chunk length of the forward pass
+    return chunkwise_tc_supported(b) && a.T > 0 && a.T % kL == 0 && a.T / kL <= kMaxSegChunks;
 }
 
 cudaError_t launch_summary(const FwdArgs &a, float *C_seg, float *n_seg, double *F_m, cudaStream_t s) {
@@ -514,6 +517,8 @@ SegPlan segment_plan(const FwdArgs &a) {
     if (G < 2) return sp;
     G = std::max(G, (NC + kMaxSegChunks - 1) / kMaxSegChunks);   // no segment longer than kMaxSegChunks
     sp.seg_chunks = (NC + G - 1) / G;
+    const int per = a.chunk / kL;   // segments hold whole chunks of the forward pass
+    sp.seg_chunks = (sp.seg_chunks + per - 1) / per * per;
     G = (NC + sp.seg_chunks - 1) / sp.seg_chunks;
     if (G < 2) return sp;
     sp.nseg = G;

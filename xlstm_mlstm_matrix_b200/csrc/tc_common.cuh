@@ -74,28 +74,32 @@ __device__ __forceinline__ float2 bf16x2_to_float2(uint32_t u) {
 }
 
 
-// V <- w V in place: 1024 16-byte chunks of a 64-token x 128-value stage, chunk
-// e in row (token) (e mod 512) / 8; 128 threads, 8 chunks each.
+// V <- w V in place: the 16L 16-byte chunks of an L-token x 128-value stage (two
+// 64-value boxes of L rows of 128 B), chunk e in row (token) (e mod 8L) / 8;
+// 128 threads, L/8 chunks each.  The 128B swizzle permutes chunks within a row,
+// so the token of a chunk does not depend on it.
 // All loads are issued before any store: the stores go to the same buffer, so
 // interleaving them would serialise every load behind the previous store.
+template <int L = 64>
 __device__ __forceinline__ void scale_v_rows(uint8_t *Vs, const float *w, int t128) {
-    uint4 u[8];
-    float ws[8];
+    constexpr int N = L / 8;
+    uint4 u[N];
+    float ws[N];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < N; ++i) {
         const int e = t128 + 128 * i;
         u[i] = *reinterpret_cast<const uint4 *>(Vs + 16 * e);
-        ws[i] = w[(e & 511) >> 3];
+        ws[i] = w[(e & (8 * L - 1)) >> 3];
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
+    for (int i = 0; i < N; ++i) {
         const float2 w2 = make_float2(ws[i], ws[i]);
         const float2 a = __fmul2_rn(bf16x2_to_float2(u[i].x), w2), b = __fmul2_rn(bf16x2_to_float2(u[i].y), w2);
         const float2 c = __fmul2_rn(bf16x2_to_float2(u[i].z), w2), d = __fmul2_rn(bf16x2_to_float2(u[i].w), w2);
         u[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(b.x, b.y), pack_bf16x2(c.x, c.y), pack_bf16x2(d.x, d.y));
     }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) *reinterpret_cast<uint4 *>(Vs + 16 * (t128 + 128 * i)) = u[i];
+    for (int i = 0; i < N; ++i) *reinterpret_cast<uint4 *>(Vs + 16 * (t128 + 128 * i)) = u[i];
 }
 
 }  // namespace
