@@ -54,9 +54,10 @@ struct SumCfg {
     static constexpr int OFF_K = 0;
     static constexpr int OFF_V = OFF_K + STAGES * K_BYTES;
     static constexpr int OFF_W = OFF_V + STAGES * V_BYTES;    // kRing x 64 weights
-    static constexpr int OFF_RED = OFF_W + kRing * kL * 4;    // 8 warps x (F, u*) doubles
-    static constexpr int OFF_F = OFF_RED + 8 * 16;            // per-chunk F offsets (doubles)
-    static constexpr int OFF_BAR = OFF_F + kMaxSegChunks * 8;
+    static constexpr int OFF_RED = OFF_W + kRing * kL * 4;    // F_seg and u* (doubles)
+    static constexpr int OFF_F = OFF_RED + 16;                // per-chunk F at the chunk's start (doubles)
+    static constexpr int OFF_UM = OFF_F + kMaxSegChunks * 8;  // per-chunk max_t (i_t - F_t), F from the chunk's start
+    static constexpr int OFF_BAR = OFF_UM + kMaxSegChunks * 8;
     // barriers: KV_FULL, KV_EMPTY, VS per stage; W_FULL, W_EMPTY per ring slot; DONE, DRAIN
     static constexpr int B_KV_FULL = 0, B_KV_EMPTY = STAGES, B_VS = 2 * STAGES, B_W_FULL = 3 * STAGES,
                          B_W_EMPTY = B_W_FULL + kRing, B_DONE = B_W_EMPTY + kRing, B_DRAIN = B_DONE + 1,
@@ -147,43 +148,64 @@ __global__ void __launch_bounds__(kSumThreads, 1)
         tmem_alloc(tmem_slot, DQK);
         tmem_relinquish();
     }
-    // F and u* of the segment: warp w scans a contiguous run of chunks, with F
-    // counted from the run's start; the runs are then joined in order.
-    const int per = (NC + 7) / 8;   // chunks per run
-    {
-        const int c0 = warp * per, c1 = min(NC, c0 + per);
-        double frun = 0.0, umax = -INFINITY;
-        float fan = 0.f, fbn = 0.f, ian = 0.f, ibn = 0.f;   // the next chunk's gates, loaded ahead
-        if (c0 < c1) {
-            const int t = kL * c0 + 2 * lane;
-            fan = fg[t]; fbn = fg[t + 1]; ian = ig[t]; ibn = ig[t + 1];
-        }
-        for (int c = c0; c < c1; ++c) {
-            const double fa = fan, fb = fbn, ia = ian, ib = ibn;
-            if (c + 1 < c1) {
-                const int t = kL * (c + 1) + 2 * lane;
-                fan = fg[t]; fbn = fg[t + 1]; ian = ig[t]; ibn = ig[t + 1];
+    // F and u* of the segment.  Pass 1: warp w takes chunks w, w + 8, ... in groups of
+    // eight, every gate load of a group issued before its first scan (one memory
+    // round trip per group, not per chunk): per chunk the total of f~ and
+    // max_t (i~_t - F_t) with F counted from the chunk's start.  Pass 2 (warp 0):
+    // the chunk totals scanned into F at each chunk's start, F_seg, and
+    // u* = max over chunks of (that maximum - F at the chunk's start).
+    double *umc = reinterpret_cast<double *>(sm + C::OFF_UM);
+    for (int c0 = warp; c0 < NC; c0 += 64) {
+        float fa[8], fb[8], ia[8], ib[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const int c = c0 + 8 * j;
+            if (c < NC) {
+                const int t = kL * c + 2 * lane;
+                fa[j] = fg[t]; fb[j] = fg[t + 1]; ia[j] = ig[t]; ib[j] = ig[t + 1];
             }
-            double excl, total;
-            chunk_scan(fa, fb, excl, total);
-            const double Fa = frun + excl + fa, Fb = Fa + fb;
-            umax = fmax(umax, fmax(ia - Fa, ib - Fb));
-            if (lane == 0) chunkF[c] = frun;
-            frun += total;
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) umax = fmax(umax, __shfl_xor_sync(0xffffffffu, umax, o));
-        if (lane == 0) { red[2 * warp] = frun; red[2 * warp + 1] = umax; }
+        for (int j = 0; j < 8; ++j) {
+            const int c = c0 + 8 * j;
+            if (c < NC) {   // warp-uniform
+                double excl, total;
+                chunk_scan(fa[j], fb[j], excl, total);
+                const double Fa = excl + fa[j], Fb = Fa + fb[j];
+                double um = fmax((double)ia[j] - Fa, (double)ib[j] - Fb);
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) um = fmax(um, __shfl_xor_sync(0xffffffffu, um, o));
+                if (lane == 0) { chunkF[c] = total; umc[c] = um; }
+            }
+        }
+    }
+    __syncthreads();
+    if (warp == 0) {   // chunk totals -> F at each chunk's start; lane l scans a contiguous run
+        const int per = (NC + 31) / 32, c0 = lane * per, c1 = min(NC, c0 + per);
+        double run = 0.0;
+        for (int c = c0; c < c1; ++c) run += chunkF[c];
+        double incl = run;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const double y = __shfl_up_sync(0xffffffffu, incl, o);
+            if (lane >= o) incl += y;
+        }
+        double f = incl - run, um = -INFINITY;
+        for (int c = c0; c < c1; ++c) {
+            const double tot = chunkF[c];
+            chunkF[c] = f;
+            um = fmax(um, umc[c] - f);
+            f += tot;
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) um = fmax(um, __shfl_xor_sync(0xffffffffu, um, o));
+        if (lane == 31) { red[0] = incl; red[1] = um; }
     }
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *tmem_slot;
-    double Fseg = 0.0, ustar = -INFINITY;
-    for (int w = 0; w < 8; ++w) {
-        ustar = fmax(ustar, red[2 * w + 1] - Fseg);
-        Fseg += red[2 * w];
-    }
+    const double Fseg = red[0], ustar = red[1];
 
     if (warp == 0) {
         // ===================== TMA producer =====================
@@ -249,8 +271,7 @@ __global__ void __launch_bounds__(kSumThreads, 1)
                 const int t = kL * (c + 2) + 2 * lane;
                 fan = fg[t]; fbn = fg[t + 1]; ian = ig[t]; ibn = ig[t + 1];
             }
-            double F0 = chunkF[c];
-            for (int w = 0; w < c / per; ++w) F0 += red[2 * w];
+            const double F0 = chunkF[c];
             if (c >= kRing && !waitw(sh, &bar[C::B_W_EMPTY + slot], ((c / kRing) - 1) & 1, kWhereSumWEmpty)) break;
             double excl, total;
             chunk_scan(fa, fb, excl, total);
@@ -268,12 +289,15 @@ __global__ void __launch_bounds__(kSumThreads, 1)
         }
     } else {
         // ===================== w V in place, n_seg; read-out of C_seg =====================
-        // Thread t128 also owns columns t128 (+ 128) of n_seg (the first value slice only).
-        constexpr int NJ = (DQK + 127) / 128;
+        // n_seg (the first value slice only): thread t128 sums 8 consecutive columns
+        // (column group cg, one 16-byte k chunk per token) over the tokens of its token
+        // group tg; the TG partial sums of a column are added once, at the end.
+        constexpr int NCG = DQK / 8, TG = 128 / NCG, TPT = kL / TG;   // column groups, token groups, tokens each
         const int t128 = tid - 128;
-        float nacc[NJ];
+        const int cg = t128 % NCG, tg = t128 / NCG;
+        float nacc[8];
 #pragma unroll
-        for (int i = 0; i < NJ; ++i) nacc[i] = 0.f;
+        for (int i = 0; i < 8; ++i) nacc[i] = 0.f;
         bool alive = true;
         for (int c = 0; c < NC; ++c) {
             const int s = c % C::STAGES, slot = c % kRing;
@@ -289,21 +313,17 @@ __global__ void __launch_bounds__(kSumThreads, 1)
             named_barrier(1, 128);
             if (t128 == 0 && alive) mbar_arrive(&bar[C::B_VS + s]);
             if (alive && slice == 0) {
-                const uint8_t *Ks = sm + C::OFF_K + s * C::K_BYTES;
+                const uint8_t *kb = sm + C::OFF_K + s * C::K_BYTES + (cg >> 3) * 8192;
+                uint4 u[TPT];
 #pragma unroll
-                for (int i = 0; i < NJ; ++i) {
-                    const int j = t128 + 128 * i;
-                    if (j < DQK) {
-                        const uint8_t *col = Ks + (j >> 6) * 8192 + (j & 7) * 2;
-                        const uint32_t chk = (j & 63) >> 3;
-                        float acc = nacc[i];
-#pragma unroll 8
-                        for (int t = 0; t < kL; ++t)
-                            acc = fmaf(w[t], __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(
-                                                 col + sw128_offset(t, chk))),
-                                       acc);
-                        nacc[i] = acc;
-                    }
+                for (int i = 0; i < TPT; ++i) u[i] = *reinterpret_cast<const uint4 *>(kb + sw128_offset(TPT * tg + i, cg & 7));
+#pragma unroll
+                for (int i = 0; i < TPT; ++i) {
+                    float x[8];
+                    unpack_bf16x8(u[i], x);
+                    const float wt = w[TPT * tg + i];
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) nacc[e] = fmaf(wt, x[e], nacc[e]);
                 }
             }
             named_barrier(1, 128);
@@ -312,14 +332,23 @@ __global__ void __launch_bounds__(kSumThreads, 1)
                 mbar_arrive(&bar[C::B_KV_EMPTY + s]);
             }
         }
+        alive = alive && waitw(sh, &bar[C::B_DONE], 0, kWhereSumDone);
+        // every k stage has been read (all updates are complete): the first one holds
+        // the TG x d_qk partial sums of n_seg
+        float *part = reinterpret_cast<float *>(sm + C::OFF_K);
         if (alive && slice == 0) {
 #pragma unroll
-            for (int i = 0; i < NJ; ++i) {
-                const int j = t128 + 128 * i;
-                if (j < DQK) p.segN[((size_t)g * p.BH + bh) * DQK + j] = nacc[i];
+            for (int e = 0; e < 8; ++e) part[tg * DQK + 8 * cg + e] = nacc[e];
+        }
+        named_barrier(1, 128);
+        if (alive && slice == 0) {
+            for (int j = t128; j < DQK; j += 128) {
+                float acc = 0.f;
+#pragma unroll
+                for (int i = 0; i < TG; ++i) acc += part[i * DQK + j];
+                p.segN[((size_t)g * p.BH + bh) * DQK + j] = acc;
             }
         }
-        alive = alive && waitw(sh, &bar[C::B_DONE], 0, kWhereSumDone);
         const int v = v0 + t128;
         if (alive && v < p.dv) {   // warp-uniform: d_v is a multiple of 64
             tc_fence_after();
