@@ -290,8 +290,9 @@ __device__ __noinline__ void exact_epilogue(uint32_t tm, uint32_t lane_base, con
 
 // Epilogue of a chunk stored as bf16 h~ (the output stage's bf16 h; the output
 // gate, if any, is applied by a separate pass): the fast and the exact chunk
-// forms.  Out of line: the plain fp32 epilogue stays compact.  Element (t, v)
-// of the chunk is at h + t * dv.
+// forms; the kernel calls it for exact chunks and stores fast ones inline.  Out
+// of line, like the fp32 exact epilogue.  Element (t, v) of the chunk is at
+// h + t * dv.
 template <class C>
 __device__ __noinline__ void bf16_epilogue(uint32_t tm, uint32_t lane_base, const float *coef, const float *inv,
                                            bool exact, __nv_bfloat16 *h, size_t dv, int len) {
@@ -939,13 +940,34 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (alive) {
                 const int len = min(kL, T - kL * c);
                 float *hc = hout + (size_t)kL * c * p.dv;
-                if (BF16H && vok) {
-                    bf16_epilogue<C>(tm, lane_base, coef_s + sb * kL, inv_s + sb * kL, exact,
-                                     static_cast<__nv_bfloat16 *>(static_cast<void *>(p.h)) +
-                                         ((size_t)bh * p.T + t_base + kL * c) * p.dv + v,
-                                     p.dv, len);
-                } else if (exact && vok) {
-                    exact_epilogue<C>(tm, lane_base, coef_s + sb * kL, inv_s + sb * kL, hc, p.dv, len);
+                if (exact && vok) {
+                    if (BF16H)
+                        bf16_epilogue<C>(tm, lane_base, coef_s + sb * kL, inv_s + sb * kL, true,
+                                         static_cast<__nv_bfloat16 *>(static_cast<void *>(p.h)) +
+                                             ((size_t)bh * p.T + t_base + kL * c) * p.dv + v,
+                                         p.dv, len);
+                    else
+                        exact_epilogue<C>(tm, lane_base, coef_s + sb * kL, inv_s + sb * kL, hc, p.dv, len);
+                } else if (vok && BF16H) {   // fast chunk, h~ stored as bf16
+                    __nv_bfloat16 *hb = static_cast<__nv_bfloat16 *>(static_cast<void *>(p.h)) +
+                                        ((size_t)bh * p.T + t_base + kL * c) * p.dv + v;
+#pragma unroll 1
+                    for (int hh = 0; hh < kL / 32; ++hh) {
+                        float rh[32], cf[32];
+                        tmem_ld32(tm + lane_base + C::TM_H + 32 * hh, rh);
+                        load32(coef_s + sb * kL + 32 * hh, cf);
+                        tmem_wait_ld();
+                        __nv_bfloat16 *hrow = hb + (size_t)32 * hh * p.dv;
+                        const int n = min(32, len - 32 * hh);
+                        if (n == 32) {
+#pragma unroll
+                            for (int x = 0; x < 32; ++x) hrow[(size_t)x * p.dv] = __float2bfloat16_rn(rh[x] * cf[x]);
+                        } else {   // the last, partial chunk of a sequence
+#pragma unroll
+                            for (int x = 0; x < 32; ++x)
+                                if (x < n) hrow[(size_t)x * p.dv] = __float2bfloat16_rn(rh[x] * cf[x]);
+                        }
+                    }
                 } else if (vok) {
 #pragma unroll 1
                     for (int hh = 0; hh < kL / 32; ++hh) {
