@@ -315,7 +315,35 @@ __global__ void bwd_dm0_kernel(const float *part, float *dm0, int BH, int slices
 
 // ---- 3. gradients of every chunk, all chunks at once ------------------------------------
 constexpr int kLd = kL + 1;   // padded row of the L x L matrices
-constexpr int kTd = 33;       // padded row of a 32-wide tile
+constexpr int kAs = 68;       // row of a 32 x 64 operand tile: 16-byte aligned, rows 4 banks apart
+
+// The block's 64 x 64 product tile, 4 x 4 outputs per thread (rows 4 ty + i, columns
+// 4 tx + j; ty = tid / 16, tx = tid % 16): acc += A^T B over the 32 rows k of the
+// K-major tiles As[k][row] and Bs[k][col].  Two 16-byte shared loads per 16 FMAs.
+__device__ __forceinline__ void tile_fma(const float *As, const float *Bs, float (&acc)[4][4], int ty, int tx) {
+#pragma unroll 8
+    for (int k = 0; k < 32; ++k) {
+        const float4 a = *reinterpret_cast<const float4 *>(As + k * kAs + 4 * ty);
+        const float4 b = *reinterpret_cast<const float4 *>(Bs + k * kAs + 4 * tx);
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[4] = {b.x, b.y, b.z, b.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+}
+__device__ __forceinline__ void zero44(float (&acc)[4][4]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+}
+// Sum over the 16 threads (tx) that share a row group: lanes l and l ^ 1, 2, 4, 8.
+__device__ __forceinline__ float sum16(float x) {
+#pragma unroll
+    for (int o = 1; o < 16; o <<= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+    return x;
+}
 
 template <typename Tin>
 __device__ __forceinline__ float ld_in(const Tin *p, size_t i) { return to_f32(p[i]); }
@@ -326,10 +354,9 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdP p) {
     float *Mm = sm;                     // [kL][kLd] M_ts
     float *Em = Mm + kL * kLd;          // [kL][kLd] E_ts
     float *Gm = Em + kL * kLd;          // [kL][kLd] S, then G_ts
-    float *tA = Gm + kL * kLd;          // [kL][kTd]
-    float *tB = tA + kL * kTd;          // [kL][kTd]
-    float *tC = tB + kL * kTd;          // [32][kTd]
-    float *sa = tC + 32 * kTd, *sz = sa + kL, *sden = sz + kL, *sds = sden + kL;
+    float *As = Gm + kL * kLd;          // [32][kAs] K-major operand tiles of the products
+    float *Bs = As + 32 * kAs;          // [32][kAs]
+    float *sa = Bs + 32 * kAs, *sz = sa + kL, *sden = sz + kL, *sds = sden + kL;
     float *sG0 = sds + kL, *sGx = sG0 + kL, *sdi = sGx + kL, *sdfi = sdi + kL, *red = sdfi + kL;
     double *su = reinterpret_cast<double *>(red + 2 * kWarps);   // [kL] u_s
     double *sFm = su + kL;                                       // [kL] F_t - m_t
@@ -393,53 +420,61 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdP p) {
     }
     __syncthreads();
 
-    const int tr = tid >> 2;          // output row (token) of this thread
-    const int cq = tid & 3;           // its quarter of the columns
-    // ---- S = Q K^T and P = DN V^T (64 x 64)
+    const int ty = tid >> 4, tx = tid & 15;   // the 4 x 4 output block of this thread
+    // Tile loaders (zero outside the chunk's L tokens and the head dims):
+    //   rows(X, ld, r0, c0, n, dst): dst[k][t] = X[t][c0 + k]   (a token-major matrix, transposed)
+    //   cols(X, ld, r0, c0, n, dst): dst[k][c] = X[r0 + k][c0 + c]
+    auto load_tok_T = [&](auto get, int c0, int ncols, float *dst) {   // dst[k][t] = get(t, c0 + k)
+        for (int e = tid; e < kL * 32; e += kThreads) {
+            const int t = e >> 5, kk = e & 31;
+            dst[kk * kAs + t] = (t < L && c0 + kk < ncols) ? get(t, c0 + kk) : 0.f;
+        }
+    };
+    auto load_rows = [&](auto get, int r0, int nrows, int c0, int ncols, float *dst) {   // dst[k][c] = get(r0 + k, c0 + c)
+        for (int e = tid; e < 32 * 64; e += kThreads) {
+            const int kk = e >> 6, c = e & 63;
+            dst[kk * kAs + c] = (r0 + kk < nrows && c0 + c < ncols) ? get(r0 + kk, c0 + c) : 0.f;
+        }
+    };
+    const auto Q = [&](int t, int j) { return p.scale * ld_in(q, (size_t)t * dqk + j); };
+    const auto Kf = [&](int t, int j) { return ld_in(k, (size_t)t * dqk + j); };
+    const auto Vf = [&](int t, int r) { return ld_in(v, (size_t)t * dv + r); };
+    const auto DN = [&](int t, int r) { return dh[(size_t)t * dv + r] / sden[t]; };
+    const auto Mf = [&](int t, int s) { return Mm[t * kLd + s]; };
+    const auto MT = [&](int t, int s) { return Mm[s * kLd + t]; };
+    const auto ET = [&](int t, int s) { return Em[s * kLd + t]; };
+
+    // ---- S = Q K^T and P = DN V^T (64 x 64), then M, E and the intra pairs' G
     {
-        float accS[16], accP[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) accS[i] = accP[i] = 0.f;
+        float accS[4][4], accP[4][4];
+        zero44(accS);
+        zero44(accP);
         for (int j0 = 0; j0 < dqk; j0 += 32) {
-            for (int e = tid; e < kL * 32; e += kThreads) {
-                const int t = e >> 5, jj = e & 31, j = j0 + jj;
-                const bool ok = t < L && j < dqk;
-                tA[t * kTd + jj] = ok ? p.scale * ld_in(q, (size_t)t * dqk + j) : 0.f;
-                tB[t * kTd + jj] = ok ? ld_in(k, (size_t)t * dqk + j) : 0.f;
-            }
             __syncthreads();
-#pragma unroll 4
-            for (int jj = 0; jj < 32; ++jj) {
-                const float a = tA[tr * kTd + jj];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) accS[i] = fmaf(a, tB[(16 * cq + i) * kTd + jj], accS[i]);
-            }
+            load_tok_T(Q, j0, dqk, As);
+            load_tok_T(Kf, j0, dqk, Bs);
             __syncthreads();
+            tile_fma(As, Bs, accS, ty, tx);
         }
         for (int r0 = 0; r0 < dv; r0 += 32) {
-            for (int e = tid; e < kL * 32; e += kThreads) {
-                const int t = e >> 5, rr = e & 31, r = r0 + rr;
-                const bool ok = t < L && r < dv;
-                tA[t * kTd + rr] = ok ? dh[(size_t)t * dv + r] / sden[t] : 0.f;
-                tB[t * kTd + rr] = ok ? ld_in(v, (size_t)t * dv + r) : 0.f;
-            }
             __syncthreads();
-#pragma unroll 4
-            for (int rr = 0; rr < 32; ++rr) {
-                const float a = tA[tr * kTd + rr];
-#pragma unroll
-                for (int i = 0; i < 16; ++i) accP[i] = fmaf(a, tB[(16 * cq + i) * kTd + rr], accP[i]);
-            }
+            load_tok_T(DN, r0, dv, As);
+            load_tok_T(Vf, r0, dv, Bs);
             __syncthreads();
+            tile_fma(As, Bs, accP, ty, tx);
         }
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-            const int s = 16 * cq + i;
-            const float w = (s <= tr && tr < L) ? expf((float)(su[s] + sFm[tr])) : 0.f;
-            const float Mv = w * (accP[i] + sds[tr]);
-            Mm[tr * kLd + s] = Mv;
-            Em[tr * kLd + s] = w * accS[i];
-            Gm[tr * kLd + s] = (s < tr) ? Mv * accS[i] : 0.f;
+        for (int i = 0; i < 4; ++i) {
+            const int t = 4 * ty + i;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int s2 = 4 * tx + j;
+                const float w = (s2 <= t && t < L) ? expf((float)(su[s2] + sFm[t])) : 0.f;
+                const float Mv = w * (accP[i][j] + sds[t]);
+                Mm[t * kLd + s2] = Mv;
+                Em[t * kLd + s2] = w * accS[i][j];
+                Gm[t * kLd + s2] = (s2 < t) ? Mv * accS[i][j] : 0.f;
+            }
         }
     }
     __syncthreads();
@@ -452,140 +487,117 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdP p) {
         sdfi[r] = acc;
     }
     // ---- dq = scale (diag(a) (DN C~_0 + ds~ n~_0^T) + M K); G_t0 = a_t q_t . (DN C~_0 + ds~ n~_0)_t
-    for (int j0 = 0; j0 < dqk; j0 += 32) {
-        float acc[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    const auto C0f = [&](int r, int j) { return C0[(size_t)r * dqk + j]; };
+    const auto Dxf = [&](int r, int j) { return Dx[(size_t)r * dqk + j]; };
+    for (int j0 = 0; j0 < dqk; j0 += 64) {
+        float acc[4][4], intra[4][4];
+        zero44(acc);
+        zero44(intra);
         for (int r0 = 0; r0 < dv; r0 += 32) {
             __syncthreads();
-            for (int e = tid; e < kL * 32; e += kThreads) {
-                const int t = e >> 5, rr = e & 31, r = r0 + rr;
-                tA[t * kTd + rr] = (t < L && r < dv) ? dh[(size_t)t * dv + r] / sden[t] : 0.f;
-            }
-            for (int e = tid; e < 32 * 32; e += kThreads) {
-                const int rr = e >> 5, jj = e & 31, r = r0 + rr, j = j0 + jj;
-                tC[rr * kTd + jj] = (r < dv && j < dqk) ? C0[(size_t)r * dqk + j] : 0.f;
-            }
+            load_tok_T(DN, r0, dv, As);
+            load_rows(C0f, r0, dv, j0, dqk, Bs);
             __syncthreads();
-#pragma unroll 4
-            for (int rr = 0; rr < 32; ++rr) {
-                const float a = tA[tr * kTd + rr];
+            tile_fma(As, Bs, acc, ty, tx);
+        }
+        for (int s0 = 0; s0 < kL; s0 += 32) {   // M K (M is zero above the diagonal and past L)
+            __syncthreads();
+            load_tok_T(Mf, s0, kL, As);
+            load_rows(Kf, s0, L, j0, dqk, Bs);
+            __syncthreads();
+            tile_fma(As, Bs, intra, ty, tx);
+        }
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(a, tC[rr * kTd + 8 * cq + i], acc[i]);
+        for (int i = 0; i < 4; ++i) {
+            const int t = 4 * ty + i;
+            float g0 = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int j = j0 + 4 * tx + jj;
+                if (t < L && j < dqk) {
+                    const float A1 = sa[t] * (acc[i][jj] + sds[t] * n0[j]);
+                    p.dq[((size_t)bh * p.T + t0 + t) * dqk + j] = p.scale * (A1 + intra[i][jj]);
+                    g0 = fmaf(Q(t, j), A1, g0);
+                }
             }
+            g0 = sum16(g0);
+            if (tx == 0) sG0[t] += g0;
         }
-        __syncthreads();
-        for (int e = tid; e < kL * 32; e += kThreads) {
-            const int t = e >> 5, jj = e & 31, j = j0 + jj;
-            const bool ok = t < L && j < dqk;
-            tA[t * kTd + jj] = ok ? p.scale * ld_in(q, (size_t)t * dqk + j) : 0.f;
-            tB[t * kTd + jj] = ok ? ld_in(k, (size_t)t * dqk + j) : 0.f;
-        }
-        __syncthreads();
-        float g0 = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int jj = 8 * cq + i, j = j0 + jj;
-            const float A1 = acc[i] + (j < dqk ? sds[tr] * n0[j] : 0.f);
-            float intra = 0.f;
-            for (int s = 0; s <= tr && s < L; ++s) intra = fmaf(Mm[tr * kLd + s], tB[s * kTd + jj], intra);
-            if (tr < L && j < dqk) p.dq[((size_t)bh * p.T + t0 + tr) * dqk + j] = p.scale * (sa[tr] * A1 + intra);
-            g0 = fmaf(tA[tr * kTd + jj], sa[tr] * A1, g0);
-        }
-        g0 += __shfl_xor_sync(0xffffffffu, g0, 1);
-        g0 += __shfl_xor_sync(0xffffffffu, g0, 2);
-        if (cq == 0) sG0[tr] += g0;
     }
     // ---- dk = M^T Q + diag(z) (V dC~_ex + 1 dn~_ex^T); di~ = k . dk; G_s,ex = k_s . (exit part)
-    for (int j0 = 0; j0 < dqk; j0 += 32) {
-        float acc[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    for (int j0 = 0; j0 < dqk; j0 += 64) {
+        float acc[4][4], intra[4][4];
+        zero44(acc);
+        zero44(intra);
         for (int r0 = 0; r0 < dv; r0 += 32) {
             __syncthreads();
-            for (int e = tid; e < kL * 32; e += kThreads) {
-                const int t = e >> 5, rr = e & 31, r = r0 + rr;
-                tA[t * kTd + rr] = (t < L && r < dv) ? ld_in(v, (size_t)t * dv + r) : 0.f;
-            }
-            for (int e = tid; e < 32 * 32; e += kThreads) {
-                const int rr = e >> 5, jj = e & 31, r = r0 + rr, j = j0 + jj;
-                tC[rr * kTd + jj] = (r < dv && j < dqk) ? Dx[(size_t)r * dqk + j] : 0.f;
-            }
+            load_tok_T(Vf, r0, dv, As);
+            load_rows(Dxf, r0, dv, j0, dqk, Bs);
             __syncthreads();
-#pragma unroll 4
-            for (int rr = 0; rr < 32; ++rr) {
-                const float a = tA[tr * kTd + rr];
+            tile_fma(As, Bs, acc, ty, tx);
+        }
+        for (int s0 = 0; s0 < kL; s0 += 32) {   // M^T Q
+            __syncthreads();
+            load_tok_T(MT, s0, kL, As);
+            load_rows(Q, s0, L, j0, dqk, Bs);
+            __syncthreads();
+            tile_fma(As, Bs, intra, ty, tx);
+        }
 #pragma unroll
-                for (int i = 0; i < 8; ++i) acc[i] = fmaf(a, tC[rr * kTd + 8 * cq + i], acc[i]);
+        for (int i = 0; i < 4; ++i) {
+            const int t = 4 * ty + i;
+            float di = 0.f, gx = 0.f;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int j = j0 + 4 * tx + jj;
+                if (t < L && j < dqk) {
+                    const float ex = sz[t] * (acc[i][jj] + dnx[j]);
+                    const float dkv = intra[i][jj] + ex;
+                    p.dk[((size_t)bh * p.T + t0 + t) * dqk + j] = dkv;
+                    const float kv = Kf(t, j);
+                    di = fmaf(kv, dkv, di);
+                    gx = fmaf(kv, ex, gx);
+                }
             }
-        }
-        __syncthreads();
-        for (int e = tid; e < kL * 32; e += kThreads) {
-            const int t = e >> 5, jj = e & 31, j = j0 + jj;
-            const bool ok = t < L && j < dqk;
-            tA[t * kTd + jj] = ok ? p.scale * ld_in(q, (size_t)t * dqk + j) : 0.f;
-            tB[t * kTd + jj] = ok ? ld_in(k, (size_t)t * dqk + j) : 0.f;
-        }
-        __syncthreads();
-        float di = 0.f, gx = 0.f;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int jj = 8 * cq + i, j = j0 + jj;
-            const float ex = sz[tr] * (acc[i] + (j < dqk ? dnx[j] : 0.f));
-            float intra = 0.f;
-            for (int s = tr; s < L; ++s) intra = fmaf(Mm[s * kLd + tr], tA[s * kTd + jj], intra);
-            const float dkv = intra + ex;
-            if (tr < L && j < dqk) p.dk[((size_t)bh * p.T + t0 + tr) * dqk + j] = dkv;
-            const float kv = tB[tr * kTd + jj];
-            di = fmaf(kv, dkv, di);
-            gx = fmaf(kv, ex, gx);
-        }
-        di += __shfl_xor_sync(0xffffffffu, di, 1);
-        di += __shfl_xor_sync(0xffffffffu, di, 2);
-        gx += __shfl_xor_sync(0xffffffffu, gx, 1);
-        gx += __shfl_xor_sync(0xffffffffu, gx, 2);
-        if (cq == 0) {
-            sdi[tr] += di;
-            sGx[tr] += gx;
+            di = sum16(di);
+            gx = sum16(gx);
+            if (tx == 0) {
+                sdi[t] += di;
+                sGx[t] += gx;
+            }
         }
     }
     // ---- dv = E^T DN + diag(z) K dC~_ex^T
-    for (int r0 = 0; r0 < dv; r0 += 32) {
-        float acc[8], ex[8];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) acc[i] = ex[i] = 0.f;
+    const auto DxT = [&](int j, int r) { return Dx[(size_t)r * dqk + j]; };
+    for (int r0 = 0; r0 < dv; r0 += 64) {
+        float ex[4][4], intra[4][4];
+        zero44(ex);
+        zero44(intra);
         for (int j0 = 0; j0 < dqk; j0 += 32) {
             __syncthreads();
-            for (int e = tid; e < kL * 32; e += kThreads) {
-                const int t = e >> 5, jj = e & 31, j = j0 + jj;
-                tB[t * kTd + jj] = (t < L && j < dqk) ? ld_in(k, (size_t)t * dqk + j) : 0.f;
-            }
-            for (int e = tid; e < 32 * 32; e += kThreads) {
-                const int rr = e >> 5, jj = e & 31, r = r0 + rr, j = j0 + jj;
-                tC[rr * kTd + jj] = (r < dv && j < dqk) ? Dx[(size_t)r * dqk + j] : 0.f;
-            }
+            load_tok_T(Kf, j0, dqk, As);
+            load_rows(DxT, j0, dqk, r0, dv, Bs);
             __syncthreads();
-#pragma unroll 4
-            for (int jj = 0; jj < 32; ++jj) {
-                const float a = tB[tr * kTd + jj];
+            tile_fma(As, Bs, ex, ty, tx);
+        }
+        for (int s0 = 0; s0 < kL; s0 += 32) {   // E^T DN
+            __syncthreads();
+            load_tok_T(ET, s0, kL, As);
+            load_rows(DN, s0, L, r0, dv, Bs);
+            __syncthreads();
+            tile_fma(As, Bs, intra, ty, tx);
+        }
 #pragma unroll
-                for (int i = 0; i < 8; ++i) ex[i] = fmaf(a, tC[(8 * cq + i) * kTd + jj], ex[i]);
+        for (int i = 0; i < 4; ++i) {
+            const int t = 4 * ty + i;
+#pragma unroll
+            for (int jj = 0; jj < 4; ++jj) {
+                const int r = r0 + 4 * tx + jj;
+                if (t < L && r < dv) p.dv_[((size_t)bh * p.T + t0 + t) * dv + r] = intra[i][jj] + sz[t] * ex[i][jj];
             }
-        }
-        __syncthreads();
-        for (int e = tid; e < kL * 32; e += kThreads) {
-            const int t = e >> 5, rr = e & 31, r = r0 + rr;
-            tA[t * kTd + rr] = (t < L && r < dv) ? dh[(size_t)t * dv + r] / sden[t] : 0.f;
-        }
-        __syncthreads();
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            const int rr = 8 * cq + i, r = r0 + rr;
-            float intra = 0.f;
-            for (int s = tr; s < L; ++s) intra = fmaf(Em[s * kLd + tr], tA[s * kTd + rr], intra);
-            if (tr < L && r < dv) p.dv_[((size_t)bh * p.T + t0 + tr) * dv + r] = intra + sz[tr] * ex[i];
         }
     }
+    __syncthreads();
     // ---- the entry state carried to the exit: G_0,ex = a_L' (<dC~_ex, C~_0> + <dn~_ex, n~_0>)
     {
         float part = 0.f;
@@ -614,8 +626,7 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdP p) {
 }
 
 size_t chunk_smem_bytes() {
-    return (size_t)(3 * kL * kLd + 2 * kL * kTd + 32 * kTd + 9 * kL + 2 * kWarps) * sizeof(float) +
-           2 * kL * sizeof(double) + 16;
+    return (size_t)(3 * kL * kLd + 2 * 32 * kAs + 9 * kL + 2 * kWarps) * sizeof(float) + 2 * kL * sizeof(double) + 16;
 }
 
 template <typename Tin>
