@@ -89,6 +89,11 @@ __global__ void __launch_bounds__(kThreads) bwd_states_kernel(BwdP p) {
     float *sdh = sv + kTok * kRows;          // [kTok][kRows] dh of the block's rows
     float *sg = sdh + kTok * kRows;          // [kTok][2] (i~, f~)
     float *sgw = sg + 2 * kTok;              // [kTok][kWarps] per-warp shares of dh . h~
+    // per-lane parts of n~ . q and of the warp's share of dh . (C~ q), [kWarps][kTok][33]: summed
+    // once per staged block of tokens (they do not feed the recurrence)
+    float *rs = sgw + kTok * kWarps;
+    float *rn = rs + kWarps * kTok * 33;
+    double *smt = reinterpret_cast<double *>(rn + kWarps * kTok * 33);   // [kTok] m_t
     const int bh = blockIdx.x / p.slices, slice = blockIdx.x % p.slices, row0 = slice * kRows;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const Tin *q = static_cast<const Tin *>(p.q) + (size_t)bh * p.T * dqk;
@@ -162,16 +167,37 @@ __global__ void __launch_bounds__(kThreads) bwd_states_kernel(BwdP p) {
                 }
                 num = fmaf(cq, qv, num);
             }
-            s = warp_sum(s);
-            num = warp_sum(num);
-            const float lower = expf((float)(-m_new));
+            rs[(warp * kTok + tt) * 33 + lane] = s;
+            rn[(warp * kTok + tt) * 33 + lane] = num;
+            if (tid == 0) smt[tt] = m_new;
+            m = m_new;
+        }
+        __syncthreads();
+        if (lane < nt) {   // token tt = lane: the lane sums, the readout's denominator, this warp's share
+            const int tt = lane, t = t0 + tt;
+            // pairwise, in the order of a butterfly reduction over the 32 lanes
+            float a[32], b[32];
+#pragma unroll
+            for (int l = 0; l < 32; ++l) {
+                a[l] = rs[(warp * kTok + tt) * 33 + l];
+                b[l] = rn[(warp * kTok + tt) * 33 + l];
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1)
+#pragma unroll
+                for (int l = 0; l < o; ++l) {
+                    a[l] += a[l + o];
+                    b[l] += b[l + o];
+                }
+            const float s = a[0], num = b[0];
+            const double mt = smt[tt];
+            const float lower = expf((float)(-mt));
             const float den = fabsf(s) > lower ? fabsf(s) : lower;
-            if (lane == 0) sgw[tt * kWarps + warp] = num / den;
-            if (slice == 0 && tid == 0) {
-                p.wmt[(size_t)bh * p.T + t] = m_new;
+            sgw[tt * kWarps + warp] = num / den;
+            if (slice == 0 && warp == 0) {
+                p.wmt[(size_t)bh * p.T + t] = mt;
                 p.wst[(size_t)bh * p.T + t] = s;
             }
-            m = m_new;
         }
         __syncthreads();
         if (tid < nt) {   // this slice's share of dh_t . h~_t
@@ -206,7 +232,7 @@ __global__ void __launch_bounds__(kThreads) bwd_adjoint_kernel(BwdP p) {
     const int dqk = p.dqk, dv = p.dv;
     float *sq = sm;                          // [kTok][dqk] scaled q
     float *sdh = sq + kTok * dqk;            // [kTok][kRows] dh_t / den~_t
-    float *ssc = sdh + kTok * kRows;         // [kTok][2] (ds~_t, f'_t)
+    float *ssc = sdh + kTok * kRows;         // [kTok][3] (ds~_t, f'_t, den~_t)
     const int bh = blockIdx.x / p.slices, slice = blockIdx.x % p.slices, row0 = slice * kRows;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const Tin *q = static_cast<const Tin *>(p.q) + (size_t)bh * p.T * dqk;
@@ -236,15 +262,15 @@ __global__ void __launch_bounds__(kThreads) bwd_adjoint_kernel(BwdP p) {
             float den, ds;
             readout_factors(st[t], mt[t], gt[t], den, ds);
             const double mp = t > 0 ? mt[t - 1] : m_init;
-            ssc[2 * tid] = ds;
-            ssc[2 * tid + 1] = expf((float)((double)fg[t] + mp - mt[t]));
+            ssc[3 * tid] = ds;
+            ssc[3 * tid + 1] = expf((float)((double)fg[t] + mp - mt[t]));
+            ssc[3 * tid + 2] = den;
         }
+        __syncthreads();
         // dh / den~ of the block's rows
         for (int e = tid; e < nt * kRows; e += kThreads) {
             const int tt = e / kRows, r = e % kRows, t = t0 + tt;
-            float den, ds;
-            readout_factors(st[t], mt[t], gt[t], den, ds);
-            sdh[e] = (row0 + r < dv) ? dh[(size_t)t * dv + row0 + r] / den : 0.f;
+            sdh[e] = (row0 + r < dv) ? dh[(size_t)t * dv + row0 + r] / ssc[3 * tt + 2] : 0.f;
         }
         __syncthreads();
         for (int tt = nt - 1; tt >= 0; --tt) {
@@ -263,7 +289,7 @@ __global__ void __launch_bounds__(kThreads) bwd_adjoint_kernel(BwdP p) {
                     if (slice == 0 && warp == 0) p.wdn[ci * dqk + j] = dn[c];
                 }
             }
-            const float ds = ssc[2 * tt], fp = ssc[2 * tt + 1];
+            const float ds = ssc[3 * tt], fp = ssc[3 * tt + 1];
             const float *qt = sq + tt * dqk;
 #pragma unroll
             for (int c = 0; c < MAXC; ++c) {
@@ -632,7 +658,8 @@ size_t chunk_smem_bytes() {
 template <typename Tin>
 cudaError_t launch_bwd_typed(BwdP p, cudaStream_t s) {
     const int maxc = (p.dqk + 31) / 32;
-    const size_t smem_seq = (size_t)(2 * kTok * p.dqk + 2 * kTok * kRows + 2 * kTok + kTok * kWarps) * sizeof(float);
+    const size_t smem_seq = (size_t)(2 * kTok * p.dqk + 2 * kTok * kRows + 2 * kTok + kTok * kWarps +
+                                     2 * kWarps * kTok * 33) * sizeof(float) + kTok * sizeof(double) + 16;
     const dim3 gseq(p.B * p.H * p.slices);
     cudaError_t e;
 #define XLSTM_BWD_SEQ(MC)                                                                              \
