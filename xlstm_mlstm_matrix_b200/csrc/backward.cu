@@ -226,8 +226,9 @@ __device__ __forceinline__ void readout_factors(float s, double m, float g, floa
 }
 
 // ---- 2. adjoints at chunk exits, backwards in t -----------------------------------------
+// Three blocks per SM up to d_qk = 256 (the register cap leaves those forms unspilled).
 template <typename Tin, int MAXC>
-__global__ void __launch_bounds__(kThreads) bwd_adjoint_kernel(BwdP p) {
+__global__ void __launch_bounds__(kThreads, MAXC <= 8 ? 3 : 1) bwd_adjoint_kernel(BwdP p) {
     extern __shared__ float sm[];
     const int dqk = p.dqk, dv = p.dv;
     float *sq = sm;                          // [kTok][dqk] scaled q
