@@ -365,6 +365,34 @@ __device__ __forceinline__ void zero44(float (&acc)[4][4]) {
 #pragma unroll
         for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
 }
+// One thread's 8 elements (e = tid + 256 i) of a 32 x 64 operand tile, fetched into
+// registers so that the next tile's global loads overlap the current tile's FMAs.
+//   TOKT: element (kk = e % 32, t = e / 32) = get(t, k0 + kk)   (token-major source, transposed)
+//   rows: element (kk = e / 64, c = e % 64) = get(k0 + kk, c0 + c)
+// Zero outside t < L, k0 + kk < nk, c0 + c < nc.
+template <bool TOKT, class G>
+__device__ __forceinline__ void fetch8(G get, int k0, int nk, int c0, int nc, int L, float (&r)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = threadIdx.x + kThreads * i;
+        if (TOKT) {
+            const int t = e >> 5, kk = e & 31;
+            r[i] = (t < L && k0 + kk < nk) ? get(t, k0 + kk) : 0.f;
+        } else {
+            const int kk = e >> 6, c = e & 63;
+            r[i] = (k0 + kk < nk && c0 + c < nc) ? get(k0 + kk, c0 + c) : 0.f;
+        }
+    }
+}
+template <bool TOKT>
+__device__ __forceinline__ void put8(float *dst, const float (&r)[8]) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int e = threadIdx.x + kThreads * i;
+        dst[TOKT ? (e & 31) * kAs + (e >> 5) : (e >> 6) * kAs + (e & 63)] = r[i];
+    }
+}
+
 // Sum over the 16 threads (tx) that share a row group: lanes l and l ^ 1, 2, 4, 8.
 __device__ __forceinline__ float sum16(float x) {
 #pragma unroll
@@ -376,7 +404,7 @@ template <typename Tin>
 __device__ __forceinline__ float ld_in(const Tin *p, size_t i) { return to_f32(p[i]); }
 
 template <typename Tin>
-__global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdP p) {
+__global__ void __launch_bounds__(kThreads, 3) bwd_chunk_kernel(BwdP p) {
     extern __shared__ float sm[];
     float *Mm = sm;                     // [kL][kLd] M_ts
     float *Em = Mm + kL * kLd;          // [kL][kLd] E_ts
@@ -448,19 +476,40 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdP p) {
     __syncthreads();
 
     const int ty = tid >> 4, tx = tid & 15;   // the 4 x 4 output block of this thread
-    // Tile loaders (zero outside the chunk's L tokens and the head dims):
-    //   rows(X, ld, r0, c0, n, dst): dst[k][t] = X[t][c0 + k]   (a token-major matrix, transposed)
-    //   cols(X, ld, r0, c0, n, dst): dst[k][c] = X[r0 + k][c0 + c]
-    auto load_tok_T = [&](auto get, int c0, int ncols, float *dst) {   // dst[k][t] = get(t, c0 + k)
-        for (int e = tid; e < kL * 32; e += kThreads) {
-            const int t = e >> 5, kk = e & 31;
-            dst[kk * kAs + t] = (t < L && c0 + kk < ncols) ? get(t, c0 + kk) : 0.f;
+    // acc += A^T B over K in 32-deep tiles, the next tile's loads in flight during the
+    // current tile's FMAs.  A[k][t] = ga(t, k) (token-major, k < na); B[k][s] = gb(s, k)
+    // (product_tt, token-major, k < nb) or B[k][c] = gb(k, c0 + c) (product_tr, k < nb,
+    // c0 + c < ncb).  Zero past the chunk's L tokens.
+    auto product_tt = [&](auto ga, int na, auto gb, int nb, int K, float (&acc)[4][4]) {
+        float ra[8], rb[8];
+        fetch8<true>(ga, 0, na, 0, 0, L, ra);
+        fetch8<true>(gb, 0, nb, 0, 0, L, rb);
+        for (int k0 = 0; k0 < K; k0 += 32) {
+            __syncthreads();
+            put8<true>(As, ra);
+            put8<true>(Bs, rb);
+            __syncthreads();
+            if (k0 + 32 < K) {
+                fetch8<true>(ga, k0 + 32, na, 0, 0, L, ra);
+                fetch8<true>(gb, k0 + 32, nb, 0, 0, L, rb);
+            }
+            tile_fma(As, Bs, acc, ty, tx);
         }
     };
-    auto load_rows = [&](auto get, int r0, int nrows, int c0, int ncols, float *dst) {   // dst[k][c] = get(r0 + k, c0 + c)
-        for (int e = tid; e < 32 * 64; e += kThreads) {
-            const int kk = e >> 6, c = e & 63;
-            dst[kk * kAs + c] = (r0 + kk < nrows && c0 + c < ncols) ? get(r0 + kk, c0 + c) : 0.f;
+    auto product_tr = [&](auto ga, int na, auto gb, int nb, int c0, int ncb, int K, float (&acc)[4][4]) {
+        float ra[8], rb[8];
+        fetch8<true>(ga, 0, na, 0, 0, L, ra);
+        fetch8<false>(gb, 0, nb, c0, ncb, L, rb);
+        for (int k0 = 0; k0 < K; k0 += 32) {
+            __syncthreads();
+            put8<true>(As, ra);
+            put8<false>(Bs, rb);
+            __syncthreads();
+            if (k0 + 32 < K) {
+                fetch8<true>(ga, k0 + 32, na, 0, 0, L, ra);
+                fetch8<false>(gb, k0 + 32, nb, c0, ncb, L, rb);
+            }
+            tile_fma(As, Bs, acc, ty, tx);
         }
     };
     const auto Q = [&](int t, int j) { return p.scale * ld_in(q, (size_t)t * dqk + j); };
@@ -476,20 +525,8 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdP p) {
         float accS[4][4], accP[4][4];
         zero44(accS);
         zero44(accP);
-        for (int j0 = 0; j0 < dqk; j0 += 32) {
-            __syncthreads();
-            load_tok_T(Q, j0, dqk, As);
-            load_tok_T(Kf, j0, dqk, Bs);
-            __syncthreads();
-            tile_fma(As, Bs, accS, ty, tx);
-        }
-        for (int r0 = 0; r0 < dv; r0 += 32) {
-            __syncthreads();
-            load_tok_T(DN, r0, dv, As);
-            load_tok_T(Vf, r0, dv, Bs);
-            __syncthreads();
-            tile_fma(As, Bs, accP, ty, tx);
-        }
+        product_tt(Q, dqk, Kf, dqk, dqk, accS);
+        product_tt(DN, dv, Vf, dv, dv, accP);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = 4 * ty + i;
@@ -520,20 +557,8 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdP p) {
         float acc[4][4], intra[4][4];
         zero44(acc);
         zero44(intra);
-        for (int r0 = 0; r0 < dv; r0 += 32) {
-            __syncthreads();
-            load_tok_T(DN, r0, dv, As);
-            load_rows(C0f, r0, dv, j0, dqk, Bs);
-            __syncthreads();
-            tile_fma(As, Bs, acc, ty, tx);
-        }
-        for (int s0 = 0; s0 < kL; s0 += 32) {   // M K (M is zero above the diagonal and past L)
-            __syncthreads();
-            load_tok_T(Mf, s0, kL, As);
-            load_rows(Kf, s0, L, j0, dqk, Bs);
-            __syncthreads();
-            tile_fma(As, Bs, intra, ty, tx);
-        }
+        product_tr(DN, dv, C0f, dv, j0, dqk, dv, acc);
+        product_tr(Mf, kL, Kf, L, j0, dqk, kL, intra);   // M K (M is zero above the diagonal and past L)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = 4 * ty + i;
@@ -556,20 +581,8 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdP p) {
         float acc[4][4], intra[4][4];
         zero44(acc);
         zero44(intra);
-        for (int r0 = 0; r0 < dv; r0 += 32) {
-            __syncthreads();
-            load_tok_T(Vf, r0, dv, As);
-            load_rows(Dxf, r0, dv, j0, dqk, Bs);
-            __syncthreads();
-            tile_fma(As, Bs, acc, ty, tx);
-        }
-        for (int s0 = 0; s0 < kL; s0 += 32) {   // M^T Q
-            __syncthreads();
-            load_tok_T(MT, s0, kL, As);
-            load_rows(Q, s0, L, j0, dqk, Bs);
-            __syncthreads();
-            tile_fma(As, Bs, intra, ty, tx);
-        }
+        product_tr(Vf, dv, Dxf, dv, j0, dqk, dv, acc);
+        product_tr(MT, kL, Q, L, j0, dqk, kL, intra);   // M^T Q
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = 4 * ty + i;
@@ -600,20 +613,8 @@ __global__ void __launch_bounds__(kThreads) bwd_chunk_kernel(BwdP p) {
         float ex[4][4], intra[4][4];
         zero44(ex);
         zero44(intra);
-        for (int j0 = 0; j0 < dqk; j0 += 32) {
-            __syncthreads();
-            load_tok_T(Kf, j0, dqk, As);
-            load_rows(DxT, j0, dqk, r0, dv, Bs);
-            __syncthreads();
-            tile_fma(As, Bs, ex, ty, tx);
-        }
-        for (int s0 = 0; s0 < kL; s0 += 32) {   // E^T DN
-            __syncthreads();
-            load_tok_T(ET, s0, kL, As);
-            load_rows(DN, s0, L, r0, dv, Bs);
-            __syncthreads();
-            tile_fma(As, Bs, intra, ty, tx);
-        }
+        product_tr(Kf, dqk, DxT, dqk, r0, dv, dqk, ex);
+        product_tr(ET, kL, DN, L, r0, dv, kL, intra);   // E^T DN
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = 4 * ty + i;
