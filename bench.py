@@ -316,7 +316,7 @@ class _Sequence:
     """One chunkwise forward over the whole batch per step (gated: through the
     output stage, bf16 o~ in and bf16 h out)."""
 
-    def __init__(self, w, inp, dev, stream, gated=False, chunk=64):
+    def __init__(self, w, inp, dev, stream, gated=False, chunk=64, kind="chunkwise"):
         import torch
         from xlstm_mlstm_matrix_b200 import capi
         self.w, self.inp, self.chunk = w, inp, chunk
@@ -348,16 +348,18 @@ class _Sequence:
             self.argv = (ctypes.byref(self.desc), ctypes.byref(self.ostage), *(P(t) for t in self.ins[:-1]),
                          *(P(t) for t in self.outs), P(self.ws), wsb, ctypes.c_void_p(stream.cuda_stream))
         else:
-            self.fn = capi.load().xlstm_mlstm_fwd_chunkwise
+            self.fn = getattr(capi.load(), "xlstm_mlstm_fwd_" + kind)
             self.argv = (ctypes.byref(self.desc), *(P(t) for t in self.ins), *(P(t) for t in self.outs),
                          P(self.ws), wsb, ctypes.c_void_p(stream.cuda_stream))
         self.stream = stream
-        self.kernel = "chunkwise (segment summaries + combine + chunkwise)" if segmented else "chunkwise"
+        if kind == "recurrent":   # one kernel, token by token; no segments
+            segmented = False
+        self.kernel = "chunkwise (segment summaries + combine + chunkwise)" if segmented else kind
         # kernels per call: the tensor-core path applies the output gate as a second, streaming pass
         self.launches = (3 if segmented else 1) + (1 if gated else 0)
         if gated:
             self.kernel += " + output gate"
-        self.name = "xlstm_mlstm_fwd_chunkwise_out" if gated else "xlstm_mlstm_fwd_chunkwise"
+        self.name = "xlstm_mlstm_fwd_chunkwise_out" if gated else "xlstm_mlstm_fwd_" + kind
 
     def step(self, i):
         st = self.fn(*self.argv)
@@ -510,41 +512,59 @@ def time_job(job, steps, warmup, stream, dev, gpu_index):
     return e0.elapsed_time(e1) / steps, clk.summary()
 
 
-# (workload, chunk length); plus the headline layer's backward
-SECONDARY = (("decode", 0), ("long_context", 64), ("long_context", 128), ("many_short", 64), ("many_short", 128))
+# (workload, chunk length or the recurrent call); plus the headline layer's backward
+FP32_PEAK_TFLOPS = 148 * 128 * 2 * 1.965e9 / 1e12   # fp32 FMA lanes x 2 FLOP x max SM clock
+SECONDARY = (("decode", 0), ("long_context", 64), ("long_context", 128), ("many_short", 64), ("many_short", 128),
+             ("many_short", "recurrent"), ("layer_7b", "recurrent"))
 
 
 def run_secondary(args, dev, stream, gpu_index):
     """The other workloads of the benchmark spec, each timed like the headline one: the
     decode step kernel (B=128 H=8 d_qk=256 d_v=512, state resident in HBM), the
-    long-context layer and the many-short-sequences layer.  One entry each with
-    its own roofline fraction; the headline value stays the 7B-like layer."""
+    long-context and many-short-sequences layers at chunk 64 and 128, and the
+    recurrent call on the many-short and 7B-like layers.  One entry each with its
+    own roofline fraction (HBM; fp32 ALU for the recurrent call); the headline
+    value stays the 7B-like layer."""
     hbm, bf16_peak, _, peak_src = peaks()
     out = []
     inp_of = {}
     for name, chunk in SECONDARY:
         if name == args.workload and chunk in (0, args.chunk):
             continue
+        kind = "recurrent" if chunk == "recurrent" else "chunkwise"
         w = workload_for_rank(name, 0)
         if name not in inp_of:
             inp_of.clear()
             inp_of[name] = make_inputs(w)
         inp = inp_of[name]
-        job = _Decode(w, inp, dev, stream) if w.steps else _Sequence(w, inp, dev, stream, chunk=chunk)
+        job = _Decode(w, inp, dev, stream) if w.steps else _Sequence(w, inp, dev, stream, chunk=chunk if
+                                                                      kind == "chunkwise" else 64, kind=kind)
         steps = min(args.steps, 100 if w.steps else 50)
         ms, clocks = time_job(job, steps, args.warmup, stream, dev, gpu_index)
         bytes_, flops = algorithmic(w)
         gbs = bytes_ / (ms * 1e-3) / 1e9
-        out.append({"workload": f"{name} L={chunk}" if chunk else name, "kernel": job.kernel, "ms_per_step": ms,
+        label = name if not chunk else (f"{name} recurrent" if kind == "recurrent" else f"{name} L={chunk}")
+        if kind == "recurrent":
+            # token by token on fp32 CUDA cores: 4 d_qk d_v + 4 d_qk FLOPs per head-token (state update
+            # and readout), against the fp32 FMA peak of 148 SMs x 128 lanes x 2 FLOP x 1965 MHz
+            rflops = w.B * w.H * w.T * (4 * w.d_qk * w.d_v + 4 * w.d_qk)
+            tf = rflops / (ms * 1e-3) / 1e12
+            roof = {"bound": "alu", "achieved": tf, "peak": FP32_PEAK_TFLOPS, "unit": "TFLOP/s",
+                    "frac": tf / FP32_PEAK_TFLOPS, "peak_source": "unit counts x max SM clock",
+                    "flops_per_launch": rflops, "hbm_frac": gbs / hbm, "traffic": None}
+        else:
+            roof = {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
+                    "frac": gbs / hbm, "peak_source": peak_src,
+                    "algorithmic_bytes_per_launch": bytes_,
+                    "traffic": traffic_for(kernel_source_sha(), w, chunk=chunk)}
+        out.append({"workload": label, "kernel": job.kernel, "ms_per_step": ms,
                     "value": tokens_per_step(w) / (ms * 1e-3), "unit": UNIT,
                     "hbm_gbs": gbs, "tflops": flops / (ms * 1e-3) / 1e12,
-                    "roofline": {"bound": "hbm", "achieved": gbs, "peak": hbm, "unit": "GB/s",
-                                 "frac": gbs / hbm, "peak_source": peak_src,
-                                 "algorithmic_bytes_per_launch": bytes_,
-                                 "traffic": traffic_for(kernel_source_sha(), w, chunk=chunk)},
+                    "roofline": roof,
                     "gpu_launches": steps * job.launches, "steps": steps, "clocks": clocks,
                     "config": config_of(w, {"l2": "working set larger than L2 (126 MB)",
-                                            **({"chunk": chunk} if chunk else {})})})
+                                            **({"chunk": chunk} if kind == "chunkwise" and chunk else {}),
+                                            **({"call": "xlstm_mlstm_fwd_recurrent"} if kind == "recurrent" else {})})})
         del job, inp
     inp_of.clear()
     # the backward of the headline sequence workload

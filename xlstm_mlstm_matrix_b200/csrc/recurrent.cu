@@ -111,14 +111,19 @@ __global__ void __launch_bounds__(kThreads) recurrent_kernel(RecP p) {
                 }
                 acc[r] = s;
             }
+            // the warp's four row sums at once: lanes trade half of their values at each
+            // of the first two steps (xor 16, then 8), then sum one value (xor 4, 2, 1);
+            // lane 8 r ends with row r
+            static_assert(kRpw == 4, "four rows per warp");
+            const bool b4 = lane & 16, b3 = lane & 8;
+            float s0 = b4 ? acc[2] : acc[0], s1 = b4 ? acc[3] : acc[1];
+            s0 += __shfl_xor_sync(0xffffffffu, b4 ? acc[0] : acc[2], 16);
+            s1 += __shfl_xor_sync(0xffffffffu, b4 ? acc[1] : acc[3], 16);
+            float rsum = b3 ? s1 : s0;
+            rsum += __shfl_xor_sync(0xffffffffu, b3 ? s0 : s1, 8);
 #pragma unroll
-            for (int r = 0; r < kRpw; ++r) acc[r] = warp_sum(acc[r]);
-            if (lane < kRpw) {
-                float val = acc[0];
-#pragma unroll
-                for (int r = 1; r < kRpw; ++r) val = (lane == r) ? acc[r] : val;
-                sh[tt * kRows + warp * kRpw + lane] = val * inv_den;
-            }
+            for (int o = 4; o > 0; o >>= 1) rsum += __shfl_xor_sync(0xffffffffu, rsum, o);
+            if ((lane & 7) == 0) sh[tt * kRows + warp * kRpw + (lane >> 3)] = rsum * inv_den;
             m = m_new;
         }
         __syncthreads();
