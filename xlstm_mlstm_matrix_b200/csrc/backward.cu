@@ -94,6 +94,7 @@ __global__ void __launch_bounds__(kThreads) bwd_states_kernel(BwdP p) {
     float *rs = sgw + kTok * kWarps;
     float *rn = rs + kWarps * kTok * 33;
     double *smt = reinterpret_cast<double *>(rn + kWarps * kTok * 33);   // [kTok] m_t
+    float *sfi = reinterpret_cast<float *>(smt + kTok);                 // [kTok][2] (f'_t, i'_t)
     const int bh = blockIdx.x / p.slices, slice = blockIdx.x % p.slices, row0 = slice * kRows;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const Tin *q = static_cast<const Tin *>(p.q) + (size_t)bh * p.T * dqk;
@@ -131,6 +132,22 @@ __global__ void __launch_bounds__(kThreads) bwd_states_kernel(BwdP p) {
             sg[2 * tid + 1] = fg[t0 + tid];
         }
         __syncthreads();
+        // the staged tokens' gates once per block: the stabilizer chain (float64) on one
+        // thread, f' and i' on one thread per token
+        if (tid == 0) {
+            double mm = m;
+            for (int tt = 0; tt < nt; ++tt) {
+                mm = fmax((double)sg[2 * tt + 1] + mm, (double)sg[2 * tt]);
+                smt[tt] = mm;
+            }
+        }
+        __syncthreads();
+        if (tid < nt) {
+            const double mp = tid ? smt[tid - 1] : m, it = sg[2 * tid], ft = sg[2 * tid + 1], mn = smt[tid];
+            sfi[2 * tid] = expf((float)(ft + mp - mn));
+            sfi[2 * tid + 1] = expf((float)(it - mn));
+        }
+        __syncthreads();
         for (int tt = 0; tt < nt; ++tt) {
             const int t = t0 + tt;
             if (t % kL == 0) {   // the stored state entering chunk t / L
@@ -148,9 +165,8 @@ __global__ void __launch_bounds__(kThreads) bwd_states_kernel(BwdP p) {
                 }
                 if (slice == 0 && tid == 0) p.wm0[ci] = m;
             }
-            const double it = sg[2 * tt], ft = sg[2 * tt + 1];
-            const double m_new = fmax(ft + m, it);
-            const float fp = expf((float)(ft + m - m_new)), ip = expf((float)(it - m_new));
+            const double m_new = smt[tt];
+            const float fp = sfi[2 * tt], ip = sfi[2 * tt + 1];
             const float *qt = sq + tt * dqk, *kt = sk + tt * dqk;
             float s = 0.f, num = 0.f;   // n~ . q and this lane's share of sum_r dh_r (C~ q)_r
 #pragma unroll
@@ -169,7 +185,6 @@ __global__ void __launch_bounds__(kThreads) bwd_states_kernel(BwdP p) {
             }
             rs[(warp * kTok + tt) * 33 + lane] = s;
             rn[(warp * kTok + tt) * 33 + lane] = num;
-            if (tid == 0) smt[tt] = m_new;
             m = m_new;
         }
         __syncthreads();
@@ -661,7 +676,7 @@ template <typename Tin>
 cudaError_t launch_bwd_typed(BwdP p, cudaStream_t s) {
     const int maxc = (p.dqk + 31) / 32;
     const size_t smem_seq = (size_t)(2 * kTok * p.dqk + 2 * kTok * kRows + 2 * kTok + kTok * kWarps +
-                                     2 * kWarps * kTok * 33) * sizeof(float) + kTok * sizeof(double) + 16;
+                                     2 * kWarps * kTok * 33 + 2 * kTok) * sizeof(float) + kTok * sizeof(double) + 16;
     const dim3 gseq(p.B * p.H * p.slices);
     cudaError_t e;
 #define XLSTM_BWD_SEQ(MC)                                                                              \

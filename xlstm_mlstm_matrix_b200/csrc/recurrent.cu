@@ -37,8 +37,8 @@ __global__ void __launch_bounds__(kThreads) recurrent_kernel(RecP p) {
     float *sq = sm;                          // [kTok][dqk] scaled q
     float *sk = sq + kTok * dqk;             // [kTok][dqk]
     float *sv = sk + kTok * dqk;             // [kTok][kRows]
-    float *sg = sv + kTok * kRows;           // [kTok][2] (i~, f~)
-    float *sh = sg + 2 * kTok;               // [kTok][kRows] outputs
+    float *sg = sv + kTok * kRows;           // [kTok][4] (f', i', e^{-m_t}, m_t) of each staged token
+    float *sh = sg + 4 * kTok;               // [kTok][kRows] outputs
 
     const int bh = blockIdx.x / p.slices;
     const int slice = blockIdx.x % p.slices;
@@ -77,15 +77,32 @@ __global__ void __launch_bounds__(kThreads) recurrent_kernel(RecP p) {
             const int tt = e / kRows, r = e % kRows;
             sv[e] = (row0 + r < dv) ? to_f32(v[(size_t)(t0 + tt) * dv + row0 + r]) : 0.f;
         }
+        if (tid < nt) {   // the gates of the staged tokens, once per block: the stabilizer chain
+            sg[4 * tid] = fg[t0 + tid];   // on one thread, the exponentials on one thread per token
+            sg[4 * tid + 1] = ig[t0 + tid];
+        }
+        __syncthreads();
+        if (tid == 0) {
+            float mm = m;
+            for (int tt = 0; tt < nt; ++tt) {
+                const float a = sg[4 * tt] + mm;
+                mm = (a > sg[4 * tt + 1]) ? a : sg[4 * tt + 1];
+                sg[4 * tt + 3] = mm;
+            }
+        }
+        __syncthreads();
         if (tid < nt) {
-            sg[2 * tid] = ig[t0 + tid];
-            sg[2 * tid + 1] = fg[t0 + tid];
+            const float mp = tid ? sg[4 * (tid - 1) + 3] : m, f = sg[4 * tid], i = sg[4 * tid + 1];
+            float m_new, fp, ip;
+            stabilized_gates(f, i, mp, m_new, fp, ip);
+            sg[4 * tid] = fp;
+            sg[4 * tid + 1] = ip;
+            sg[4 * tid + 2] = expf(-m_new);
         }
         __syncthreads();
 
         for (int tt = 0; tt < nt; ++tt) {
-            float m_new, fp, ip;
-            stabilized_gates(sg[2 * tt + 1], sg[2 * tt], m, m_new, fp, ip);
+            const float fp = sg[4 * tt], ip = sg[4 * tt + 1], lower = sg[4 * tt + 2], m_new = sg[4 * tt + 3];
             const float *qt = sq + tt * dqk, *kt = sk + tt * dqk;
             float qv[MAXC], kv[MAXC];
             float nq = 0.f;
@@ -98,7 +115,7 @@ __global__ void __launch_bounds__(kThreads) recurrent_kernel(RecP p) {
                 nq += n[c] * qv[c];
             }
             nq = warp_sum(nq);
-            const float inv_den = 1.f / fmaxf(fabsf(nq), expf(-m_new));
+            const float inv_den = 1.f / fmaxf(fabsf(nq), lower);
             float acc[kRpw];
 #pragma unroll
             for (int r = 0; r < kRpw; ++r) {
@@ -155,7 +172,7 @@ template <typename Tin>
 cudaError_t launch_typed(const RecP &p, int dqk, cudaStream_t s) {
     const int slices = p.slices;
     dim3 grid(p.B * p.H * slices);
-    const size_t smem = (size_t)(2 * kTok * dqk + 2 * kTok * kRows + 2 * kTok) * sizeof(float);
+    const size_t smem = (size_t)(2 * kTok * dqk + 2 * kTok * kRows + 4 * kTok) * sizeof(float);
     const int maxc = (dqk + 31) / 32;
 #define XLSTM_REC_CASE(MC)                                                                   \
     if (maxc <= MC) {                                                                        \
