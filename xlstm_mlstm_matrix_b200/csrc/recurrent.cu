@@ -7,8 +7,10 @@
 //
 // A block owns kRows rows of C~ for one (batch, head): warp w holds rows
 // [w*kRpw, (w+1)*kRpw) in registers, lane l holds columns l, l+32, ... of each.
-// Every warp keeps the whole normaliser n~ (its own lanes' columns) so that
-// n~^T q is a warp reduction and no block barrier sits on the per-token path.
+// The normaliser n~ is spread over the block, thread i holding columns i, i+256,
+// ...: per token each thread stores its part of n~^T q, and the staged tokens'
+// sums and denominators are formed once per staged block, when the outputs are
+// written, so no block barrier sits on the per-token path.
 // Inputs for kTok tokens are staged in shared memory per barrier; the outputs
 // of those tokens are staged too and written back as contiguous rows.
 #include "common.cuh"
@@ -38,7 +40,9 @@ __global__ void __launch_bounds__(kThreads) recurrent_kernel(RecP p) {
     float *sk = sq + kTok * dqk;             // [kTok][dqk]
     float *sv = sk + kTok * dqk;             // [kTok][kRows]
     float *sg = sv + kTok * kRows;           // [kTok][4] (f', i', e^{-m_t}, m_t) of each staged token
-    float *sh = sg + 4 * kTok;               // [kTok][kRows] outputs
+    float *sh = sg + 4 * kTok;               // [kTok][kRows] outputs (before the denominator)
+    float *snq = sh + kTok * kRows;          // [kTok][kThreads] parts of n~^T q
+    float *sden = snq + kTok * kThreads;     // [kTok] 1 / max(|n~^T q|, e^{-m_t})
 
     const int bh = blockIdx.x / p.slices;
     const int slice = blockIdx.x % p.slices;
@@ -51,13 +55,18 @@ __global__ void __launch_bounds__(kThreads) recurrent_kernel(RecP p) {
     const float *ig = p.ig + (size_t)bh * p.T;
     const float *fg = p.fg + (size_t)bh * p.T;
 
+    constexpr int NJ = (MAXC * 32 + kThreads - 1) / kThreads;   // normaliser columns per thread
     float C[kRpw][MAXC];
-    float n[MAXC];
+    float n[NJ];
     float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < NJ; ++i) {
+        const int j = tid + kThreads * i;
+        n[i] = (p.n0 && j < dqk) ? p.n0[(size_t)bh * dqk + j] : 0.f;
+    }
 #pragma unroll
     for (int c = 0; c < MAXC; ++c) {
         const int j = lane + 32 * c;
-        n[c] = (p.n0 && j < dqk) ? p.n0[(size_t)bh * dqk + j] : 0.f;
 #pragma unroll
         for (int r = 0; r < kRpw; ++r) {
             const int row = row0 + warp * kRpw + r;
@@ -105,17 +114,22 @@ __global__ void __launch_bounds__(kThreads) recurrent_kernel(RecP p) {
             const float fp = sg[4 * tt], ip = sg[4 * tt + 1], lower = sg[4 * tt + 2], m_new = sg[4 * tt + 3];
             const float *qt = sq + tt * dqk, *kt = sk + tt * dqk;
             float qv[MAXC], kv[MAXC];
-            float nq = 0.f;
 #pragma unroll
             for (int c = 0; c < MAXC; ++c) {
                 const int j = lane + 32 * c;
                 qv[c] = (j < dqk) ? qt[j] : 0.f;
                 kv[c] = (j < dqk) ? kt[j] : 0.f;
-                n[c] = fp * n[c] + ip * kv[c];
-                nq += n[c] * qv[c];
             }
-            nq = warp_sum(nq);
-            const float inv_den = 1.f / fmaxf(fabsf(nq), lower);
+            float nq = 0.f;   // this thread's part of n~^T q
+#pragma unroll
+            for (int i = 0; i < NJ; ++i) {
+                const int j = tid + kThreads * i;
+                if (j < dqk) {
+                    n[i] = fp * n[i] + ip * kt[j];
+                    nq += n[i] * qt[j];
+                }
+            }
+            snq[tt * kThreads + tid] = nq;
             float acc[kRpw];
 #pragma unroll
             for (int r = 0; r < kRpw; ++r) {
@@ -140,14 +154,26 @@ __global__ void __launch_bounds__(kThreads) recurrent_kernel(RecP p) {
             rsum += __shfl_xor_sync(0xffffffffu, b3 ? s0 : s1, 8);
 #pragma unroll
             for (int o = 4; o > 0; o >>= 1) rsum += __shfl_xor_sync(0xffffffffu, rsum, o);
-            if ((lane & 7) == 0) sh[tt * kRows + warp * kRpw + (lane >> 3)] = rsum * inv_den;
+            if ((lane & 7) == 0) sh[tt * kRows + warp * kRpw + (lane >> 3)] = rsum;
             m = m_new;
+        }
+        __syncthreads();
+        {   // n~^T q of each staged token: 16 threads per token, 16 parts each, then a 16-lane sum
+            const int tt = tid >> 4, part = tid & 15;
+            float x = 0.f;
+            if (tt < nt) {
+#pragma unroll
+                for (int i = 0; i < kThreads / 16; ++i) x += snq[tt * kThreads + part + 16 * i];
+            }
+#pragma unroll
+            for (int o = 8; o > 0; o >>= 1) x += __shfl_xor_sync(0xffffffffu, x, o);
+            if (part == 0 && tt < nt) sden[tt] = 1.f / fmaxf(fabsf(x), sg[4 * tt + 2]);
         }
         __syncthreads();
         float *h = p.h + ((size_t)bh * p.T + t0) * dv + row0;
         for (int e = tid; e < nt * kRows; e += kThreads) {
             const int tt = e / kRows, r = e % kRows;
-            if (row0 + r < dv) h[(size_t)tt * dv + r] = sh[e];
+            if (row0 + r < dv) h[(size_t)tt * dv + r] = sh[e] * sden[tt];
         }
     }
 
@@ -163,7 +189,11 @@ __global__ void __launch_bounds__(kThreads) recurrent_kernel(RecP p) {
                 if (row < dv) p.C1[((size_t)bh * dv + row) * dqk + j] = C[r][c];
             }
         }
-        if (p.n1 && slice == 0 && warp == 0) p.n1[(size_t)bh * dqk + j] = n[c];
+    }
+#pragma unroll
+    for (int i = 0; i < NJ; ++i) {
+        const int j = tid + kThreads * i;
+        if (p.n1 && slice == 0 && j < dqk) p.n1[(size_t)bh * dqk + j] = n[i];
     }
     if (p.m1 && slice == 0 && tid == 0) p.m1[bh] = m;
 }
@@ -172,7 +202,7 @@ template <typename Tin>
 cudaError_t launch_typed(const RecP &p, int dqk, cudaStream_t s) {
     const int slices = p.slices;
     dim3 grid(p.B * p.H * slices);
-    const size_t smem = (size_t)(2 * kTok * dqk + 2 * kTok * kRows + 4 * kTok) * sizeof(float);
+    const size_t smem = (size_t)(2 * kTok * dqk + 2 * kTok * kRows + 4 * kTok + kTok * kThreads + kTok) * sizeof(float);
     const int maxc = (dqk + 31) / 32;
 #define XLSTM_REC_CASE(MC)                                                                   \
     if (maxc <= MC) {                                                                        \
