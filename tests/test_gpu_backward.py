@@ -84,6 +84,8 @@ SHAPES = [  # B, H, T, dqk, dv, dtype, state, dstate
     (1, 1, 200, 32, 48, "f32", True, True),
     (2, 2, 1, 16, 16, "bf16", True, True),
     (1, 1, 333, 64, 128, "bf16", False, True),
+    (1, 1, 70, 512, 32, "f32", True, True),    # the largest head dim the ABI takes
+    (1, 1, 65, 384, 48, "bf16", True, False),
 ]
 
 

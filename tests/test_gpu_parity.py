@@ -42,6 +42,11 @@ SMALL = [  # B, H, T, dqk, dv
     (1, 1, 65, 64, 384),
     (2, 1, 130, 128, 192),
     (3, 2, 71, 256, 320),
+    # the largest head dims the ABI takes, and odd ones (CUDA-core kernels; more than one
+    # normaliser column per thread in the recurrent kernel)
+    (1, 1, 70, 512, 32),
+    (1, 2, 40, 384, 48),
+    (2, 1, 33, 80, 16),
 ]
 TC_SHAPES = [sh for sh in SMALL if sh[3] in (64, 128, 256) and sh[4] % 64 == 0]
 
@@ -173,8 +178,9 @@ def test_composition_across_calls(dtype, dv):
 
 
 @pytest.mark.parametrize("dtype", ["f32", "bf16"])
-def test_step_matches_oracle_and_recurrent(dtype):
-    B, H, T, dqk, dv = 3, 2, 40, 64, 96
+@pytest.mark.parametrize("dqk,dv", [(64, 96), (512, 32), (80, 48)])
+def test_step_matches_oracle_and_recurrent(dtype, dqk, dv):
+    B, H, T = 3, 2, 40
     inp = small_inputs(B, H, T, dqk, dv, dtype, True, seed=21)
     ref = oracle_sequence(inp)
     C = to_dev(inp["C0"], "f32"); n = to_dev(inp["n0"], "f32"); m = to_dev(inp["m0"], "f32")
