@@ -47,7 +47,8 @@
 // 32 KB P tile fill the rest), loaded once the previous chunk's update is done.
 //
 // Warps: 0 TMA producer (and L2 prefetch two chunks ahead), 1 MMA issuer (owns
-// TMEM), 2 gate scan, 3 normaliser,
+// TMEM), 2 gate scan, 3 normaliser (warps 0 and 3 swap roles at L = 128 and at
+// d_qk = 256),
 // 4-7 state group (the first columns of the state split, n.q, epilogue), 8-11
 // token group (w V, the other columns of the state split, P).
 // Every wait is bounded: one that gives up records XLSTM_ERR_TIMEOUT in the
@@ -65,6 +66,7 @@ namespace {
 using namespace sm100;
 
 constexpr int kDvs = 128;           // value rows per block
+
 constexpr int kThreads = 384;
 constexpr int kNG = 4;              // gate-ring slots
 constexpr double kRescale = 20.0;   // gauge drift allowed before the state is rescaled
@@ -519,6 +521,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                     const __grid_constant__ CUtensorMap tmv, const TcParams p) {
     using C = Cfg<DQK, L>;
     constexpr int kL = L;
+    // The normaliser runs on warp 0 (SMSP 0) and the TMA producer on warp 3 where that
+    // measured faster: at L = 128 the P pass of rows 96-127 (four column groups, warp 11)
+    // shares SMSP 3 with warp 3; at d_qk = 256 the normaliser is the longest of the
+    // single-warp roles.  Otherwise the other way round.
+    constexpr bool kSwap = L == 128 || DQK == 256;
+    constexpr int kWarpTma = kSwap ? 3 : 0, kWarpNorm = kSwap ? 0 : 3;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *sm = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t *bar = reinterpret_cast<uint64_t *>(sm + C::OFF_BAR);
@@ -567,7 +575,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t tm = *tmem_slot;
     uint8_t *Ps = sm + C::OFF_P;
 
-    if (warp == 0) {
+    if (warp == kWarpTma) {
         // ===================== TMA producer =====================
         // Order per chunk: k, q, then v.  With one V stage (L = 128) the v copy waits
         // for the previous chunk's update, and k and q of the chunk must not queue
@@ -798,7 +806,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             __syncwarp();
             if (lane == 0 && !(p.fault == 1 && c == 1)) mbar_arrive(&bar[B_G_FULL + slot]);
         }
-    } else if (warp == 3) {
+    } else if (warp == kWarpNorm) {
         // ===================== normaliser n_acc =====================
         constexpr int NPL = DQK / 32;             // columns per lane
         const int j0 = lane * NPL;
