@@ -374,6 +374,12 @@ __device__ __forceinline__ void tile_fma(const float *As, const float *Bs, float
             for (int j = 0; j < 4; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
     }
 }
+__device__ __forceinline__ void zero48(float (&acc)[4][8]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+}
 __device__ __forceinline__ void zero44(float (&acc)[4][4]) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
@@ -408,6 +414,41 @@ __device__ __forceinline__ void put8(float *dst, const float (&r)[8]) {
     }
 }
 
+// 64 x 128 product tile, 4 x 8 outputs per thread: rows 4 ty + i, columns 4 tx + j and
+// 64 + 4 tx + j (two groups of four, so each 16-byte load of a quarter-warp is contiguous).
+// B is a K-major 32 x 128 tile with rows kBs floats apart.
+constexpr int kBs = 132;
+__device__ __forceinline__ void tile_fma_w(const float *As, const float *Bs, float (&acc)[4][8], int ty, int tx) {
+#pragma unroll 4
+    for (int k = 0; k < 32; ++k) {
+        const float4 a = *reinterpret_cast<const float4 *>(As + k * kAs + 4 * ty);
+        const float4 b0 = *reinterpret_cast<const float4 *>(Bs + k * kBs + 4 * tx);
+        const float4 b1 = *reinterpret_cast<const float4 *>(Bs + k * kBs + 64 + 4 * tx);
+        const float av[4] = {a.x, a.y, a.z, a.w}, bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+}
+// One thread's 16 elements (e = tid + 256 i) of a 32 x 128 row-major operand tile:
+// element (kk = e / 128, c = e % 128) = get(k0 + kk, c0 + c), zero outside k0 + kk < nk, c0 + c < nc.
+template <class G>
+__device__ __forceinline__ void fetch16(G get, int k0, int nk, int c0, int nc, float (&r)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int e = threadIdx.x + kThreads * i, kk = e >> 7, c = e & 127;
+        r[i] = (k0 + kk < nk && c0 + c < nc) ? get(k0 + kk, c0 + c) : 0.f;
+    }
+}
+__device__ __forceinline__ void put16(float *dst, const float (&r)[16]) {
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+        const int e = threadIdx.x + kThreads * i;
+        dst[(e >> 7) * kBs + (e & 127)] = r[i];
+    }
+}
+
 // Sum over the 16 threads (tx) that share a row group: lanes l and l ^ 1, 2, 4, 8.
 __device__ __forceinline__ float sum16(float x) {
 #pragma unroll
@@ -419,14 +460,14 @@ template <typename Tin>
 __device__ __forceinline__ float ld_in(const Tin *p, size_t i) { return to_f32(p[i]); }
 
 template <typename Tin>
-__global__ void __launch_bounds__(kThreads, 3) bwd_chunk_kernel(BwdP p) {
+__global__ void __launch_bounds__(kThreads, 2) bwd_chunk_kernel(BwdP p) {
     extern __shared__ float sm[];
     float *Mm = sm;                     // [kL][kLd] M_ts
     float *Em = Mm + kL * kLd;          // [kL][kLd] E_ts
     float *Gm = Em + kL * kLd;          // [kL][kLd] S, then G_ts
     float *As = Gm + kL * kLd;          // [32][kAs] K-major operand tiles of the products
-    float *Bs = As + 32 * kAs;          // [32][kAs]
-    float *sa = Bs + 32 * kAs, *sz = sa + kL, *sden = sz + kL, *sds = sden + kL;
+    float *Bs = As + 32 * kAs;          // [32][kBs] (64-wide tiles use the first kAs-strided rows)
+    float *sa = Bs + 32 * kBs, *sz = sa + kL, *sden = sz + kL, *sds = sden + kL;
     float *sG0 = sds + kL, *sGx = sG0 + kL, *sdi = sGx + kL, *sdfi = sdi + kL, *red = sdfi + kL;
     double *su = reinterpret_cast<double *>(red + 2 * kWarps);   // [kL] u_s
     double *sFm = su + kL;                                       // [kL] F_t - m_t
@@ -511,6 +552,23 @@ __global__ void __launch_bounds__(kThreads, 3) bwd_chunk_kernel(BwdP p) {
             tile_fma(As, Bs, acc, ty, tx);
         }
     };
+    // 64 x 128 output tiles (B row-major, 128 columns from c0)
+    auto product_trw = [&](auto ga, int na, auto gb, int nb, int c0, int ncb, int K, float (&acc)[4][8]) {
+        float ra[8], rb[16];
+        fetch8<true>(ga, 0, na, 0, 0, L, ra);
+        fetch16(gb, 0, nb, c0, ncb, rb);
+        for (int k0 = 0; k0 < K; k0 += 32) {
+            __syncthreads();
+            put8<true>(As, ra);
+            put16(Bs, rb);
+            __syncthreads();
+            if (k0 + 32 < K) {
+                fetch8<true>(ga, k0 + 32, na, 0, 0, L, ra);
+                fetch16(gb, k0 + 32, nb, c0, ncb, rb);
+            }
+            tile_fma_w(As, Bs, acc, ty, tx);
+        }
+    };
     auto product_tr = [&](auto ga, int na, auto gb, int nb, int c0, int ncb, int K, float (&acc)[4][4]) {
         float ra[8], rb[8];
         fetch8<true>(ga, 0, na, 0, 0, L, ra);
@@ -568,19 +626,19 @@ __global__ void __launch_bounds__(kThreads, 3) bwd_chunk_kernel(BwdP p) {
     // ---- dq = scale (diag(a) (DN C~_0 + ds~ n~_0^T) + M K); G_t0 = a_t q_t . (DN C~_0 + ds~ n~_0)_t
     const auto C0f = [&](int r, int j) { return C0[(size_t)r * dqk + j]; };
     const auto Dxf = [&](int r, int j) { return Dx[(size_t)r * dqk + j]; };
-    for (int j0 = 0; j0 < dqk; j0 += 64) {
-        float acc[4][4], intra[4][4];
-        zero44(acc);
-        zero44(intra);
-        product_tr(DN, dv, C0f, dv, j0, dqk, dv, acc);
-        product_tr(Mf, kL, Kf, L, j0, dqk, kL, intra);   // M K (M is zero above the diagonal and past L)
+    for (int j0 = 0; j0 < dqk; j0 += 128) {
+        float acc[4][8], intra[4][8];
+        zero48(acc);
+        zero48(intra);
+        product_trw(DN, dv, C0f, dv, j0, dqk, dv, acc);
+        product_trw(Mf, kL, Kf, L, j0, dqk, kL, intra);   // M K (M is zero above the diagonal and past L)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = 4 * ty + i;
             float g0 = 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int j = j0 + 4 * tx + jj;
+            for (int jj = 0; jj < 8; ++jj) {
+                const int j = j0 + 64 * (jj >> 2) + 4 * tx + (jj & 3);
                 if (t < L && j < dqk) {
                     const float A1 = sa[t] * (acc[i][jj] + sds[t] * n0[j]);
                     p.dq[((size_t)bh * p.T + t0 + t) * dqk + j] = p.scale * (A1 + intra[i][jj]);
@@ -592,19 +650,19 @@ __global__ void __launch_bounds__(kThreads, 3) bwd_chunk_kernel(BwdP p) {
         }
     }
     // ---- dk = M^T Q + diag(z) (V dC~_ex + 1 dn~_ex^T); di~ = k . dk; G_s,ex = k_s . (exit part)
-    for (int j0 = 0; j0 < dqk; j0 += 64) {
-        float acc[4][4], intra[4][4];
-        zero44(acc);
-        zero44(intra);
-        product_tr(Vf, dv, Dxf, dv, j0, dqk, dv, acc);
-        product_tr(MT, kL, Q, L, j0, dqk, kL, intra);   // M^T Q
+    for (int j0 = 0; j0 < dqk; j0 += 128) {
+        float acc[4][8], intra[4][8];
+        zero48(acc);
+        zero48(intra);
+        product_trw(Vf, dv, Dxf, dv, j0, dqk, dv, acc);
+        product_trw(MT, kL, Q, L, j0, dqk, kL, intra);   // M^T Q
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = 4 * ty + i;
             float di = 0.f, gx = 0.f;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int j = j0 + 4 * tx + jj;
+            for (int jj = 0; jj < 8; ++jj) {
+                const int j = j0 + 64 * (jj >> 2) + 4 * tx + (jj & 3);
                 if (t < L && j < dqk) {
                     const float ex = sz[t] * (acc[i][jj] + dnx[j]);
                     const float dkv = intra[i][jj] + ex;
@@ -624,18 +682,18 @@ __global__ void __launch_bounds__(kThreads, 3) bwd_chunk_kernel(BwdP p) {
     }
     // ---- dv = E^T DN + diag(z) K dC~_ex^T
     const auto DxT = [&](int j, int r) { return Dx[(size_t)r * dqk + j]; };
-    for (int r0 = 0; r0 < dv; r0 += 64) {
-        float ex[4][4], intra[4][4];
-        zero44(ex);
-        zero44(intra);
-        product_tr(Kf, dqk, DxT, dqk, r0, dv, dqk, ex);
-        product_tr(ET, kL, DN, L, r0, dv, kL, intra);   // E^T DN
+    for (int r0 = 0; r0 < dv; r0 += 128) {
+        float ex[4][8], intra[4][8];
+        zero48(ex);
+        zero48(intra);
+        product_trw(Kf, dqk, DxT, dqk, r0, dv, dqk, ex);
+        product_trw(ET, kL, DN, L, r0, dv, kL, intra);   // E^T DN
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
             const int t = 4 * ty + i;
 #pragma unroll
-            for (int jj = 0; jj < 4; ++jj) {
-                const int r = r0 + 4 * tx + jj;
+            for (int jj = 0; jj < 8; ++jj) {
+                const int r = r0 + 64 * (jj >> 2) + 4 * tx + (jj & 3);
                 if (t < L && r < dv) p.dv_[((size_t)bh * p.T + t0 + t) * dv + r] = intra[i][jj] + sz[t] * ex[i][jj];
             }
         }
@@ -669,7 +727,8 @@ __global__ void __launch_bounds__(kThreads, 3) bwd_chunk_kernel(BwdP p) {
 }
 
 size_t chunk_smem_bytes() {
-    return (size_t)(3 * kL * kLd + 2 * 32 * kAs + 9 * kL + 2 * kWarps) * sizeof(float) + 2 * kL * sizeof(double) + 16;
+    return (size_t)(3 * kL * kLd + 32 * kAs + 32 * kBs + 9 * kL + 2 * kWarps) * sizeof(float) + 2 * kL * sizeof(double) +
+           16;
 }
 
 template <typename Tin>
