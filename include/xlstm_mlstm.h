@@ -102,11 +102,11 @@ typedef struct {
  *                      (desc) bytes a long sequence with few heads runs as
  *                      parallel segments.  Calls sharing a workspace must not
  *                      overlap on the device.
- * Chunk lengths: 0 (= 64) and 64 for both input types; 16 and 32 for fp32
- * inputs only; 128 for bf16 inputs with d_qk = 64 or 128 and d_v a multiple
- * of 64 (the shapes the tensor-core kernel takes).  Every other length (256
- * among them), 16 or 32 with bf16 inputs, and 128 at d_qk = 256 return
- * XLSTM_ERR_UNSUPPORTED: the tensor-core kernel that runs bf16 inputs holds
+ * Chunk lengths: 0 (= 64) and 64 for both input types; 16, 32 and 128 for
+ * fp32 inputs (CUDA-core kernel); 128 for bf16 inputs with d_qk = 64 or 128
+ * and d_v a multiple of 64 (the shapes the tensor-core kernel takes).  Every
+ * other length (256 among them), 16 or 32 with bf16 inputs, and bf16 128 at
+ * d_qk = 256 return XLSTM_ERR_UNSUPPORTED: the tensor-core kernel that runs bf16 inputs holds
  * the state, its readout copy and one chunk's S and H accumulators in tensor
  * memory (512 columns), which at d_qk = 256 fits a chunk of 64 tokens only, and
  * at L = 256 no d_qk.  The chunk length is an evaluation order, not part of the

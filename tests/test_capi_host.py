@@ -138,10 +138,10 @@ def test_workspace_and_chunk_rules(lib):
         # "tcgen05" on a GPU (the driver's tensor-map encoder); not "none" anywhere
         d = capi.make_desc(1, 1, 4, dqk, 64, capi.XLSTM_BF16, 1.0, L)
         assert capi.xlstm_mlstm_chunkwise_kernel(d) != "none", (dqk, L)
-    # fp32 inputs: the CUDA-core kernel takes 16, 32 and 64
-    for L in (16, 32, 64):
+    # fp32 inputs: the CUDA-core kernel takes 16, 32, 64 and 128
+    for L in (16, 32, 64, 128):
         assert capi.xlstm_mlstm_chunkwise_kernel(capi.make_desc(1, 1, 4, 64, 64, capi.XLSTM_F32, 1.0, L)) == "simt"
-    for L in (128, 256):
+    for L in (48, 256):
         d = capi.make_desc(1, 1, 4, 64, 64, capi.XLSTM_F32, 1.0, L)
         assert call(d) == capi.XLSTM_ERR_UNSUPPORTED, L
 

@@ -78,7 +78,7 @@ def test_tensor_core_path_selected():
 def test_chunk_size_invariance(dv):
     """The chunk length is an evaluation order, not part of the method (the pages
     give no chunkwise form): every supported length must give the recurrence's
-    result.  fp32 inputs run on the CUDA-core kernel at L in {16, 32, 64}; bf16
+    result.  fp32 inputs run on the CUDA-core kernel at L in {16, 32, 64, 128}; bf16
     inputs run on the tensor-core kernel at L in {64, 128} (checked against the
     oracle and against each other), and are compared with the CUDA-core kernel at
     L in {16, 32} on the same (bf16-exact) values."""
@@ -86,10 +86,10 @@ def test_chunk_size_invariance(dv):
     bf = small_inputs(2, 2, 203, 64, dv, "bf16", True, seed=3)
     outs = {}
     ref_f = oracle_sequence(f32)
-    for L in (16, 32, 64):
+    for L in (16, 32, 64, 128):
         outs[L] = gpu_sequence(f32, "chunkwise", chunk=L)
         compare(outs[L], ref_f, "f32", f"fp32 L={L}")
-    for L in (16, 32):
+    for L in (16, 32, 128):
         mx, _ = inputs.relative_errors(outs[L][0], outs[64][0])
         assert mx <= 1e-4, f"fp32 chunk {L} vs 64: {mx:.2e}"
     B, H, T, dqk = bf["q"].shape

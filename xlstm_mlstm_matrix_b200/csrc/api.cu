@@ -36,7 +36,7 @@ bool dims_ok(const xlstm_mlstm_desc_t *d) {
 
 size_t elem(const xlstm_mlstm_desc_t *d) { return d->qkv_dtype == XLSTM_BF16 ? 2 : 4; }
 
-// Chunk lengths each path takes: 64 for every input type; 16 and 32 for fp32
+// Chunk lengths each path takes: 64 for every input type; 16, 32 and 128 for fp32
 // inputs, which run on the CUDA-core kernel; 128 for bf16 inputs with d_qk <= 128
 // on the tensor-core kernel (tensor memory holds the state, its readout copy and
 // one chunk's S and H; at d_qk = 256 only L = 64 fits).  Other lengths are
@@ -44,7 +44,7 @@ size_t elem(const xlstm_mlstm_desc_t *d) { return d->qkv_dtype == XLSTM_BF16 ? 2
 bool chunk_ok(const xlstm_mlstm_desc_t *d) {
     const int L = d->chunk ? d->chunk : 64;
     if (L == 64) return true;
-    if (d->qkv_dtype == XLSTM_F32) return L == 16 || L == 32;
+    if (d->qkv_dtype == XLSTM_F32) return L == 16 || L == 32 || L == 128;
     if (L != 128) return false;
     xlstm::FwdArgs a{};
     a.dtype = d->qkv_dtype; a.chunk = L; a.T = 1; a.dqk = d->d_qk; a.dv = d->d_v;

@@ -237,6 +237,7 @@ cudaError_t launch_typed(const ChunkP &p, cudaStream_t s) {
         case 16: return launch_L<Tin, 16>(p, s);
         case 32: return launch_L<Tin, 32>(p, s);
         case 64: return launch_L<Tin, 64>(p, s);
+        case 128: return launch_L<Tin, 128>(p, s);
         default: return cudaErrorInvalidValue;
     }
 }
