@@ -21,13 +21,13 @@ from xlstm_mlstm_matrix_b200 import capi, inputs
 pytestmark = pytest.mark.gpu
 
 
-def _run(entry, w, tensors, ws=None):
+def _run(entry, w, tensors, ws=None, chunk=64):
     q, k, v, ig, fg, C0, n0, m0 = tensors
     h = torch.empty(w.B, w.H, w.T, w.d_v, device="cuda")
     C1 = torch.empty(w.B, w.H, w.d_v, w.d_qk, device="cuda")
     n1 = torch.empty(w.B, w.H, w.d_qk, device="cuda")
     m1 = torch.empty(w.B, w.H, device="cuda")
-    desc = capi.make_desc(w.B, w.H, w.T, w.d_qk, w.d_v, capi.XLSTM_BF16, w.d_qk ** -0.5, 64)
+    desc = capi.make_desc(w.B, w.H, w.T, w.d_qk, w.d_v, capi.XLSTM_BF16, w.d_qk ** -0.5, chunk)
     if ws is None:
         st = entry(desc, q, k, v, ig, fg, C0, n0, m0, h, C1, n1, m1)
     else:
@@ -49,15 +49,15 @@ def _case(d_qk, d_v):
     return w, inp, tensors, ws
 
 
-@pytest.mark.parametrize("d_qk,d_v", [(256, 512), (128, 128)])
-def test_noalloc_matches_oracle_and_workspace_entry_twice(d_qk, d_v):
+@pytest.mark.parametrize("d_qk,d_v,chunk", [(256, 512, 64), (128, 128, 64), (128, 128, 128)])
+def test_noalloc_matches_oracle_and_workspace_entry_twice(d_qk, d_v, chunk):
     assert torch.cuda.is_available(), "needs a CUDA device"
     capi.load()
     w, inp, tensors, ws = _case(d_qk, d_v)
-    ref = _run(capi.xlstm_mlstm_fwd_chunkwise, w, tensors, ws)
+    ref = _run(capi.xlstm_mlstm_fwd_chunkwise, w, tensors, ws, chunk=chunk)
     oracle_ref = oracle_sequence(inp)
     for i in range(2):   # the shared scratch keeps the previous call's contents
-        got = _run(capi.xlstm_mlstm_fwd_chunkwise_noalloc, w, tensors)
+        got = _run(capi.xlstm_mlstm_fwd_chunkwise_noalloc, w, tensors, chunk=chunk)
         assert capi.xlstm_mlstm_noalloc_status() == (capi.XLSTM_OK, 0)
         compare(got, oracle_ref, "bf16", f"noalloc call {i} against the oracle")
         for name, a, b in zip(("h", "C", "n", "m"), got, ref):
