@@ -60,6 +60,8 @@
 #include "tc_common.cuh"
 #include "tma_host.cuh"
 
+#include <mutex>
+
 namespace xlstm {
 namespace {
 
@@ -160,6 +162,7 @@ struct TcParams {
     float *h, *C1, *n1, *m1;
     int32_t *status;
     int fault;
+    int block0;   // index of this launch's first block in the whole grid (a split launch)
 };
 
 // Entry state of segment seg of sequence bh: the caller's (or none: zero state,
@@ -540,9 +543,10 @@ __global__ void __launch_bounds__(kThreads, 1)
     float *coef_s = inv_s + 2 * kL;                            // [2][L] AH_t/den_t
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int slice = blockIdx.x % p.nslices;
-    const int seg = (blockIdx.x / p.nslices) % p.nseg;
-    const int bh = blockIdx.x / (p.nslices * p.nseg);
+    const int blk = (int)blockIdx.x + p.block0;
+    const int slice = blk % p.nslices;
+    const int seg = (blk / p.nslices) % p.nseg;
+    const int bh = blk / (p.nslices * p.nseg);
     const int v0 = slice * kDvs;
     const int t_base = p.seg_len * seg;                    // first token of this block's segment
     const int T = min(p.T - t_base, p.seg_len);            // tokens in the segment
@@ -1135,6 +1139,43 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
 }
 
+// Blocks of the first launch when a grid of nblk one-per-SM blocks ends in a partial
+// wave: every block before that wave, rounded down to whole sequences (per_seq blocks
+// each, so that their h~ is one contiguous range).  0: no split (one wave or less,
+// whole waves, not one sequence before the last wave, or more than four blocks' h~
+// for each SM the last wave leaves idle: their gate would outlast that wave).
+int overlap_split(int nblk, int per_seq) {
+    const int nsm = sm_count();
+    if (nsm <= 0 || nblk <= nsm || nblk % nsm == 0) return 0;
+    const int first = (nblk - nblk % nsm) / per_seq * per_seq;
+    const int idle = nsm - (nblk - first);
+    return first >= per_seq && idle >= 1 && first <= 4 * idle ? first : 0;
+}
+
+// The second stream of a split launch and its two events, one set per device, made on
+// first use and kept; the mutex keeps the record / wait sequence of one call from
+// interleaving with another's.
+struct OverlapStreams {
+    std::mutex mu;
+    cudaStream_t side = nullptr;
+    cudaEvent_t first = nullptr, gated = nullptr;
+    bool ok = false;
+};
+OverlapStreams *overlap_streams() {
+    constexpr int kMaxDev = 64;
+    static OverlapStreams sets[kMaxDev];
+    static std::once_flag once[kMaxDev];
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return nullptr;
+    OverlapStreams &o = sets[dev];
+    std::call_once(once[dev], [&o] {
+        o.ok = cudaStreamCreateWithFlags(&o.side, cudaStreamNonBlocking) == cudaSuccess &&
+               cudaEventCreateWithFlags(&o.first, cudaEventDisableTiming) == cudaSuccess &&
+               cudaEventCreateWithFlags(&o.gated, cudaEventDisableTiming) == cudaSuccess;
+    });
+    return o.ok ? &o : nullptr;
+}
+
 template <int DQK, int L>
 cudaError_t launch_dqk(const FwdArgs &a, cudaStream_t s, int fault) {
     using C = Cfg<DQK, L>;
@@ -1164,11 +1205,40 @@ cudaError_t launch_dqk(const FwdArgs &a, cudaStream_t s, int fault) {
     auto kern = a.out.h_bf16 ? chunk_tc_kernel<DQK, L, true> : chunk_tc_kernel<DQK, L, false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
     if (e != cudaSuccess) return e;
-    kern<<<BH * p.nseg * p.nslices, kThreads, C::SMEM, s>>>(tq, tk, tv, p);
+    const int nblk = BH * p.nseg * p.nslices, per_seq = p.nseg * p.nslices;
+    const int split = a.out.o ? overlap_split(nblk, per_seq) : 0;
+    OverlapStreams *ov = split ? overlap_streams() : nullptr;
+    p.block0 = 0;
+    if (!ov) {
+        kern<<<nblk, kThreads, C::SMEM, s>>>(tq, tk, tv, p);
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+        // the output gate as one streaming pass over h~ in place
+        if (a.out.o) return launch_output_gate(a.out, a.h, (size_t)BH * a.T * a.dv, s);
+        return cudaSuccess;
+    }
+    // The output gate of the blocks before the last, partial wave runs on the SMs that
+    // wave leaves idle: blocks [0, split), then the rest, on the caller's stream; a
+    // second stream waits for the first blocks and gates their h~ with one block on
+    // each idle SM, blocks that no block of the rest can share (whichever of the two
+    // launches is placed first, the rest find their SMs); the caller's stream waits
+    // for that gate and gates the rest's h~.
+    std::lock_guard<std::mutex> lock(ov->mu);
+    const size_t nA = (size_t)(split / per_seq) * a.T * a.dv, nAll = (size_t)BH * a.T * a.dv;
+    kern<<<split, kThreads, C::SMEM, s>>>(tq, tk, tv, p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    // the output gate as one streaming pass over h~ in place
-    if (a.out.o) return launch_output_gate(a.out, a.h, (size_t)BH * a.T * a.dv, s);
-    return cudaSuccess;
+    if ((e = cudaEventRecord(ov->first, s)) != cudaSuccess) return e;
+    p.block0 = split;
+    kern<<<nblk - split, kThreads, C::SMEM, s>>>(tq, tk, tv, p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(ov->side, ov->first, 0)) != cudaSuccess) return e;
+    if ((e = launch_output_gate_on_sms(a.out, a.h, nA, ov->side, sm_count() - (nblk - split))) != cudaSuccess)
+        return e;
+    if ((e = cudaEventRecord(ov->gated, ov->side)) != cudaSuccess) return e;
+    if ((e = cudaStreamWaitEvent(s, ov->gated, 0)) != cudaSuccess) return e;
+    const size_t hb = a.out.h_bf16 ? 2 : 4, ob = a.out.o_bf16 ? 2 : 4;
+    OutStage rest = a.out;
+    rest.o = static_cast<const char *>(a.out.o) + nA * ob;
+    return launch_output_gate(rest, reinterpret_cast<char *>(a.h) + nA * hb, nAll - nA, s);
 }
 
 }  // namespace

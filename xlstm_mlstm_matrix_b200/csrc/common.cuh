@@ -75,7 +75,12 @@ bool chunkwise_tc_shape_ok(const FwdArgs &a);     // shapes the tensor-core kern
 bool chunkwise_tc_supported(const FwdArgs &a);    // ... and the driver's TMA encoder is available
 cudaError_t launch_chunkwise_tc(const FwdArgs &a, cudaStream_t s);
 // h <- sigmoid(o~) h~ over n elements in place (h in the output stage's dtype).
+int sm_count();   // SMs of the current device (first call's device; 148 if the query fails)
+// The output gate over n elements of h~ in place (n a multiple of 8, 16-byte aligned
+// pointers): a grid-strided streaming pass over every SM; _on_sms: on nsm SMs only,
+// one block each that no other block shares, beside a kernel that holds the rest.
 cudaError_t launch_output_gate(const OutStage &os, void *h, size_t n, cudaStream_t s);
+cudaError_t launch_output_gate_on_sms(const OutStage &os, void *h, size_t n, cudaStream_t s, int nsm);
 void set_chunkwise_tc_fault(int mode);   // test hook: applies to the next launch only
 
 // ---- small device helpers ------------------------------------------------

@@ -443,17 +443,6 @@ __global__ void __launch_bounds__(kCombineThreads) seg_combine_kernel(const Comb
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
-int sm_count() {
-    static int n = 0;
-    if (!n) {
-        int dev = 0, v = 0;
-        n = (cudaGetDevice(&dev) == cudaSuccess &&
-             cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
-                ? v
-                : 148;
-    }
-    return n;
-}
 
 template <int DQK>
 cudaError_t launch_summaries_dqk(const FwdArgs &a, const SegPlan &sp, cudaStream_t s) {
@@ -532,6 +521,18 @@ cudaError_t launch_combine(int BH, int dv, int dqk, int nsum, const float *C0, c
     const int n4 = (dv * dqk + dqk) / 4;
     seg_combine_kernel<<<dim3((n4 + kCombineThreads - 1) / kCombineThreads, BH), kCombineThreads, 0, s>>>(q);
     return cudaGetLastError();
+}
+
+int sm_count() {
+    static int n = 0;
+    if (!n) {
+        int dev = 0, v = 0;
+        n = (cudaGetDevice(&dev) == cudaSuccess &&
+             cudaDeviceGetAttribute(&v, cudaDevAttrMultiProcessorCount, dev) == cudaSuccess && v > 0)
+                ? v
+                : 148;
+    }
+    return n;
 }
 
 SegPlan segment_plan(const FwdArgs &a) {
