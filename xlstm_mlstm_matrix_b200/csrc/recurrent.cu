@@ -111,7 +111,7 @@ __global__ void __launch_bounds__(kThreads) recurrent_kernel(RecP p) {
         __syncthreads();
 
         for (int tt = 0; tt < nt; ++tt) {
-            const float fp = sg[4 * tt], ip = sg[4 * tt + 1], lower = sg[4 * tt + 2], m_new = sg[4 * tt + 3];
+            const float fp = sg[4 * tt], ip = sg[4 * tt + 1], m_new = sg[4 * tt + 3];
             const float *qt = sq + tt * dqk, *kt = sk + tt * dqk;
             float qv[MAXC], kv[MAXC];
 #pragma unroll
