@@ -128,18 +128,13 @@ struct Cfg {
     static constexpr int NBARS = 48;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM = OFF_MISC + 64 + 1024;          // + alignment slack
+    static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t TM_C = 0;
     static constexpr uint32_t TM_CHI = DQK;
     static constexpr uint32_t TM_CLO = DQK + DQK / 2;          // unused when BIG
     static constexpr uint32_t TM_H = BIG ? DQK + DQK / 2 : 2 * DQK;
     static constexpr uint32_t TM_S = TM_H + L;                 // S, or the intra part of an exact chunk
-    // tensor-memory columns allocated (a power of two): 256 when the state, its readout
-    // copy and one chunk's S and H fit (d_qk = 64, L = 64), and then two blocks share an SM
-    static constexpr uint32_t TMEM_COLS = TM_S + L <= 256 ? 256 : 512;
     static_assert(TM_S + L <= TMEM_COLS, "tensor memory budget");
-    // blocks per SM: two when tensor memory, shared memory (228 KB per SM, 1 KB of it
-    // reserved per block) and 80 registers a thread allow; the kernel's launch bounds
-    static constexpr int CTAS = TMEM_COLS == 256 && 2 * (SMEM + 1024) <= 233472 ? 2 : 1;
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -524,7 +519,7 @@ __device__ __forceinline__ void split_range(uint32_t tm, uint32_t lane_base, int
 // BF16H: h~ is stored as bf16 (the output stage's bf16 h); the plain
 // instantiation keeps the fp32 store path alone.
 template <int DQK, int L, bool BF16H>
-__global__ void __launch_bounds__(kThreads, Cfg<DQK, L>::CTAS)
+__global__ void __launch_bounds__(kThreads, 1)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const TcParams p) {
     using C = Cfg<DQK, L>;
@@ -1209,11 +1204,9 @@ cudaError_t launch_dqk(const FwdArgs &a, cudaStream_t s, int fault) {
     }
     auto kern = a.out.h_bf16 ? chunk_tc_kernel<DQK, L, true> : chunk_tc_kernel<DQK, L, false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
-    if (e == cudaSuccess && C::CTAS > 1)   // room for both blocks' shared memory
-        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     const int nblk = BH * p.nseg * p.nslices, per_seq = p.nseg * p.nslices;
-    const int split = a.out.o && C::CTAS == 1 ? overlap_split(nblk, per_seq) : 0;
+    const int split = a.out.o ? overlap_split(nblk, per_seq) : 0;
     OverlapStreams *ov = split ? overlap_streams() : nullptr;
     p.block0 = 0;
     if (!ov) {
