@@ -92,20 +92,26 @@ def test_plain_call_unchanged_by_null_output_stage():
     assert torch.equal(h0, h1) and all(torch.equal(a, b) for a, b in zip(st0, st1))
 
 
-def test_gated_output_split_launch():
+@pytest.mark.parametrize("o_dtype,h_dtype", [("bf16", "bf16"), ("f32", "bf16"), ("bf16", "f32"), ("f32", "f32")])
+def test_gated_output_split_launch(o_dtype, h_dtype):
     """More blocks than SMs with a partial last wave: the call splits its grid in two
     launches and gates the first launch's h~ while the second runs.  Against the
-    oracle, and element for element against the ungated call's bf16 h~ gated here."""
+    oracle, and element for element against the ungated call's h~ (in h's dtype) gated
+    here."""
     sms = torch.cuda.get_device_properties(0).multi_processor_count
     heads = sms // 4 + 3          # 4 blocks per head (d_v = 512): a partial second wave
     inp = small_inputs(1, heads, 130, 64, 512, "bf16", True, seed=29)
-    got, o_np = run(inp, "bf16", "bf16")
-    compare(got, reference(inp, o_np), "bf16", "gated split launch")
-    plain, _ = run(inp, "bf16", "bf16", gate=False)
+    got, o_np = run(inp, o_dtype, h_dtype)
+    compare(got, reference(inp, o_np), "bf16", f"gated split launch, o {o_dtype} h {h_dtype}")
+    plain, _ = run(inp, o_dtype, h_dtype, gate=False)
     o = torch.from_numpy(o_np.astype(np.float32))
     h_tilde = torch.from_numpy(plain[0])
-    want = (h_tilde / (1.0 + torch.exp(-o))).to(torch.bfloat16).float().numpy()
-    # one bf16 unit of the larger of the two where the exponentials round differently
-    np.testing.assert_allclose(got[0], want, rtol=2 ** -7, atol=1e-30)
+    gated = h_tilde / (1.0 + torch.exp(-o))
+    if h_dtype == "bf16":
+        # one bf16 unit of the larger of the two where the exponentials round differently
+        want, rtol = gated.to(torch.bfloat16).float().numpy(), 2 ** -7
+    else:
+        want, rtol = gated.numpy(), 1e-6
+    np.testing.assert_allclose(got[0], want, rtol=rtol, atol=1e-30)
     for a, b in zip(got[1:], plain[1:]):
         assert np.array_equal(a, b)
