@@ -128,13 +128,18 @@ struct Cfg {
     static constexpr int NBARS = 48;
     static constexpr int OFF_MISC = OFF_BAR + NBARS * 8;
     static constexpr int SMEM = OFF_MISC + 64 + 1024;          // + alignment slack
-    static constexpr uint32_t TMEM_COLS = 512;
     static constexpr uint32_t TM_C = 0;
     static constexpr uint32_t TM_CHI = DQK;
     static constexpr uint32_t TM_CLO = DQK + DQK / 2;          // unused when BIG
     static constexpr uint32_t TM_H = BIG ? DQK + DQK / 2 : 2 * DQK;
     static constexpr uint32_t TM_S = TM_H + L;                 // S, or the intra part of an exact chunk
+    // tensor-memory columns allocated (a power of two): 256 when the state, its readout
+    // copy and one chunk's S and H fit (d_qk = 64, L = 64), and then two blocks share an SM
+    static constexpr uint32_t TMEM_COLS = TM_S + L <= 256 ? 256 : 512;
     static_assert(TM_S + L <= TMEM_COLS, "tensor memory budget");
+    // blocks per SM: two when tensor memory, shared memory (228 KB per SM, 1 KB of it
+    // reserved per block) and 80 registers a thread allow; the kernel's launch bounds
+    static constexpr int CTAS = TMEM_COLS == 256 && 2 * (SMEM + 1024) <= 233472 ? 2 : 1;
     static_assert(SMEM <= 232448, "shared memory budget");
 };
 
@@ -148,7 +153,13 @@ enum : int {
     // B_VT: w V is in place for a fast chunk (token group); B_VT_EXACT: the gauge
     // move and w V of an exact chunk are done (state group).  Two producers on one
     // barrier could complete two phases before the MMA warp waits for the first.
-    B_S_FULL = B_G_EMPTY + kNG, B_S_EMPTY, B_OPS, B_VT, B_VT_EXACT, B_CONV0, B_CONV1, B_CLO_FREE, B_H_FULL, B_H_EMPTY,
+    // B_OPS (P and the row sums of chunk c) and, with two V stages, B_VT come in pairs
+    // indexed by the chunk's parity: the phase for chunk c+2 cannot complete before
+    // each consumer has waited for chunk c's (it needs a later hand-off of that
+    // consumer: the epilogue of c, or the update of c), where one barrier's phase for
+    // c+1 could.
+    B_S_FULL = B_G_EMPTY + kNG, B_S_EMPTY, B_OPS, B_VT = B_OPS + 2, B_VT_EXACT = B_VT + 2, B_CONV0, B_CONV1,
+    B_CLO_FREE, B_H_FULL, B_H_EMPTY,
     B_UPD_DONE, B_N_READY, B_N_FREE = B_N_READY + 2, B_DRAIN = B_N_FREE + 2, B_COUNT
 };
 static_assert(B_COUNT <= 48, "barrier space");
@@ -519,7 +530,7 @@ __device__ __forceinline__ void split_range(uint32_t tm, uint32_t lane_base, int
 // BF16H: h~ is stored as bf16 (the output stage's bf16 h); the plain
 // instantiation keeps the fp32 store path alone.
 template <int DQK, int L, bool BF16H>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, Cfg<DQK, L>::CTAS)
     chunk_tc_kernel(const __grid_constant__ CUtensorMap tmq, const __grid_constant__ CUtensorMap tmk,
                     const __grid_constant__ CUtensorMap tmv, const TcParams p) {
     using C = Cfg<DQK, L>;
@@ -561,8 +572,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(&bar[B_N_READY + i], 1); mbar_init(&bar[B_N_FREE + i], 1);
         }
         for (int i = 0; i < kNG; ++i) { mbar_init(&bar[B_G_FULL + i], 1); mbar_init(&bar[B_G_EMPTY + i], 3); }
-        const int ones[] = {B_S_FULL, B_S_EMPTY, B_OPS, B_VT, B_VT_EXACT, B_CONV1, B_CLO_FREE, B_H_FULL, B_H_EMPTY,
-                            B_UPD_DONE, B_DRAIN};
+        const int ones[] = {B_S_FULL, B_S_EMPTY, B_OPS, B_OPS + 1, B_VT, B_VT + 1, B_VT_EXACT, B_CONV1, B_CLO_FREE,
+                            B_H_FULL, B_H_EMPTY, B_UPD_DONE, B_DRAIN};
         mbar_init(&bar[B_CONV0], 2);   // both compute groups split half of the state
         for (int b : ones) mbar_init(&bar[b], 1);
         *sh.abort_flag = 0;
@@ -634,7 +645,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t idU = make_idesc(128, DQK, kFmtBF16, kFmtBF16, 1, 1);
             const uint32_t p_addr = smem_u32(Ps), clo_addr = smem_u32(sm + C::OFF_CLO);
             bool issued = false, prev_exact = false;
-            int nfast = 0, nexact = 0;   // phases of B_VT and B_VT_EXACT consumed
+            int nfast = 0, nexact = 0;   // phases of B_VT (one V stage) and B_VT_EXACT consumed
             for (int c = 0; c < NC; ++c) {
                 const int s = c & 1, slot = c % kNG, sv = C::VST == 2 ? s : 0;
                 const uint32_t vph = C::VST == 2 ? (c >> 1) & 1 : c & 1;   // phase of V_FULL
@@ -662,12 +673,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (!wait1(sh, &bar[B_G_FULL + slot], (c / kNG) & 1, kWhereMmaGate)) break;
                 const bool exact = gring[slot * C::G_FLOATS + C::G_SCAL + kSExact] != 0.f;
                 if (!wait1(sh, &bar[B_CONV0], c & 1, kWhereMmaConv)) break;
-                // Two V stages: w V(c) is waited here, not before the intra part: the token
-                // group's next phase of B_VT (chunk c+1) may complete during the readout, and
-                // a wait for the earlier phase after that would never return.  One V stage:
-                // V(c+1) cannot land before this chunk's update, so the wait moves to the
-                // intra part.
-                if (C::VST == 2 && !exact && !wait1(sh, &bar[B_VT], (nfast++) & 1, kWhereMmaVt)) break;
+                // Two V stages: w V(c) is waited here, before the readout, on the barrier of
+                // c's parity, which the token group completes once per chunk (exact chunks
+                // included, unscaled); it scales V(c+1) during the readout and V(c+2) only
+                // after this chunk's update.  One V stage: V(c+1) cannot land before this
+                // chunk's update, so the wait moves to the intra part.
+                if (C::VST == 2 && !exact && !wait1(sh, &bar[B_VT + (c & 1)], (c >> 1) & 1, kWhereMmaVt)) break;
                 if (c >= 1 && !prev_exact && !wait1(sh, &bar[B_H_EMPTY], (c - 1) & 1, kWhereMmaHEmpty)) break;
                 tc_fence_after();
                 // H = C_hi Q^T + C_lo Q^T
@@ -699,8 +710,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 // intra part: fast chunks accumulate (w V)^T (mask S)^T onto H; exact
                 // chunks put V^T P^T into the S columns
                 // P(c) is needed only from here: the C Q^T MMAs above overlap its computation
-                // (B_OPS cannot run a phase ahead: P(c+1) needs S(c+1), issued after this chunk)
-                if (!wait1(sh, &bar[B_OPS], c & 1, kWhereMmaOps)) break;
+                // (P(c+2) needs S(c+2), issued after this chunk)
+                if (!wait1(sh, &bar[B_OPS + (c & 1)], (c >> 1) & 1, kWhereMmaOps)) break;
                 if (!wait1(sh, &bar[B_V_FULL + sv], vph, kWhereMmaKvFull)) break;
                 if (C::VST == 1 && !exact && !wait1(sh, &bar[B_VT], (nfast++) & 1, kWhereMmaVt)) break;
                 tc_fence_after();
@@ -927,8 +938,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 mbar_arrive(&bar[B_Q_EMPTY + s]);
                 mbar_arrive(&bar[B_N_FREE + s]);
             }
-            // --- denominators, once the token group has published the row sums
-            alive = alive && waitw(sh, &bar[B_OPS], c & 1, kWhereStOps);
+            // --- denominators, once the token group has published the row sums (P(c+2),
+            //     the next phase of this barrier, needs S(c+2), which the MMA warp issues
+            //     only after the readout of c+1 has waited for this chunk's epilogue)
+            alive = alive && waitw(sh, &bar[B_OPS + (c & 1)], (c >> 1) & 1, kWhereStOps);
             if (alive && st < kL) {
                 const float inv = 1.f / fmaxf(fabsf(nq_s[sb * kL + st] + rs_s[sb * kL + st]), g[C::G_LOWER + st]);
                 inv_s[sb * kL + st] = inv;
@@ -1083,7 +1096,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             named_barrier(2, 128);
             if (tk == 0 && alive) {
                 mbar_arrive(&bar[B_S_EMPTY]);
-                mbar_arrive(&bar[B_OPS]);
+                mbar_arrive(&bar[B_OPS + (c & 1)]);
                 if (C::VST == 2) mbar_arrive(&bar[B_G_EMPTY + slot]);
             }
             if (C::VST == 1) {   // --- fast chunk: V(c) <- w V(c) in place, before the intra product
@@ -1113,9 +1126,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (C::VST == 2 && c + 1 < NC) {
                 const int j = c + 1, sj = j & 1, slot_j = j % kNG;
                 const float *gj = gring + slot_j * C::G_FLOATS;
-                // the MMA warp waits for w V(c) right after the split of chunk c: scaling V(c+1)
-                // only after that split keeps the two phases of B_VT from both completing
-                // before the MMA warp has waited for the first
+                // the MMA warp waits for w V(c) right after the split of chunk c; V(c+1) is
+                // scaled after that split (its barrier is the other one of the pair)
                 if (c >= 0) alive = alive && waitw(sh, &bar[B_CONV0], c & 1, kWhereTkConv);
                 alive = alive && waitw(sh, &bar[B_G_FULL + slot_j], (j / kNG) & 1, kWhereTkGate);
                 const bool ex = alive && gj[C::G_SCAL + kSExact] != 0.f;
@@ -1126,7 +1138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     fence_proxy_async_smem();
                 }
                 named_barrier(2, 128);   // unconditional: every warp of the group takes every barrier
-                if (tk == 0 && alive && !ex) mbar_arrive(&bar[B_VT]);
+                if (tk == 0 && alive) mbar_arrive(&bar[B_VT + (j & 1)]);
             }
             if (c == -1) named_barrier(3, 256);   // C_acc is initialised before either group splits it
         }
@@ -1204,9 +1216,11 @@ cudaError_t launch_dqk(const FwdArgs &a, cudaStream_t s, int fault) {
     }
     auto kern = a.out.h_bf16 ? chunk_tc_kernel<DQK, L, true> : chunk_tc_kernel<DQK, L, false>;
     e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM);
+    if (e == cudaSuccess && C::CTAS > 1)   // room for both blocks' shared memory
+        e = cudaFuncSetAttribute(kern, cudaFuncAttributePreferredSharedMemoryCarveout, cudaSharedmemCarveoutMaxShared);
     if (e != cudaSuccess) return e;
     const int nblk = BH * p.nseg * p.nslices, per_seq = p.nseg * p.nslices;
-    const int split = a.out.o ? overlap_split(nblk, per_seq) : 0;
+    const int split = a.out.o && C::CTAS == 1 ? overlap_split(nblk, per_seq) : 0;
     OverlapStreams *ov = split ? overlap_streams() : nullptr;
     p.block0 = 0;
     if (!ov) {
