@@ -1,0 +1,56 @@
+"""The chunkwise kernel's barrier hand-offs (model in barrier_protocol.py): no
+deadlock and no phase overrun for every chunk count, V-stage count, head size class
+and pattern of exact chunks tried; and the earlier forms are rejected: one B_OPS and
+one B_VT barrier with two V stages, and the token group waiting for an exact chunk's
+V with one V stage (a consumer could come to wait for a phase after the next one
+had completed)."""
+import itertools
+
+import pytest
+
+from barrier_protocol import chunkwise_protocol
+
+PATTERNS = [(), (0,), (1,), (0, 1), (2, 3, 5), (1, 3, 5, 7), tuple(range(9))]
+
+
+@pytest.mark.parametrize("vst,big", [(2, False), (2, True), (1, False)])
+@pytest.mark.parametrize("nc", [1, 2, 3, 6, 9])
+def test_protocol_has_no_deadlock_or_overrun(vst, big, nc):
+    for exact in PATTERNS:
+        ex = tuple(c for c in exact if c < nc)
+        problems = chunkwise_protocol(nc, vst, big, ex).check()
+        assert not problems, (vst, big, nc, ex, problems[:3])
+
+
+@pytest.mark.parametrize("big", [False, True])
+def test_single_ops_and_vt_barriers_are_rejected(big):
+    """With one B_OPS the state group's wait for P(c) can be overtaken; with one B_VT
+    the MMA warp's wait for w V(c) can, except at d_qk = 256, where the token group
+    scales V(c+1) only after the MMA warp has freed the C_lo tile of chunk c."""
+    found = set()
+    for nc, exact in itertools.product([3, 6], [(), (2,), (1, 4)]):
+        for p in chunkwise_protocol(nc, 2, big, tuple(c for c in exact if c < nc), paired=False).check():
+            assert p.startswith("overrun"), p
+            found.add(p.split(":")[1].split()[0])
+    assert found == ({"OPS"} if big else {"OPS", "VT"}), found
+
+
+def test_exact_chunk_v_wait_with_one_v_stage_is_rejected():
+    problems = chunkwise_protocol(3, 1, False, (1,), exact_v_wait=True).check()
+    assert any(p.startswith("overrun: V_FULL") for p in problems), problems
+
+
+def test_checker_finds_a_missing_arrival():
+    """A planted defect: the state group never releases H (B_H_EMPTY)."""
+    P = chunkwise_protocol(3, 2, False)
+    P.roles["state"] = [op for op in P.roles["state"] if op[1] != "H_EMPTY"]
+    assert any(p.startswith("deadlock") for p in P.check())
+
+
+def test_checker_finds_an_underrun():
+    """A planted defect: with one V stage and chunk 1 exact, a token group that no
+    longer waits for S, the update or H could start waiting for V(2) while V(1),
+    which it skipped, is still in flight."""
+    P = chunkwise_protocol(4, 1, False, (1,))
+    P.roles["token"] = [op for op in P.roles["token"] if op[1] not in ("S_FULL", "UPD_DONE", "H_FULL")]
+    assert any(p.startswith("underrun: the wait of token for V_FULL") for p in P.check())

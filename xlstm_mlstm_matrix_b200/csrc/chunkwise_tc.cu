@@ -1100,7 +1100,12 @@ __global__ void __launch_bounds__(kThreads, Cfg<DQK, L>::CTAS)
                 if (C::VST == 2) mbar_arrive(&bar[B_G_EMPTY + slot]);
             }
             if (C::VST == 1) {   // --- fast chunk: V(c) <- w V(c) in place, before the intra product
-                alive = alive && waitw(sh, &bar[B_V_FULL], c & 1, kWhereTkKv);
+                // An exact chunk's V is not touched here, and not waited for either: nothing
+                // would hold V(c+1) back until this wait (the MMA warp's update, which frees
+                // the stage, waits only for the state group then), so its phase could be
+                // overtaken.  A later wait for a fast chunk's V stays exact: V(c') has landed
+                // by then up to c'-1 (S(c') follows the update of c'-1) and not beyond c'.
+                if (!exact) alive = alive && waitw(sh, &bar[B_V_FULL], c & 1, kWhereTkKv);
                 if (alive && !exact) {
                     scale_v_rows<kL>(sm + C::OFF_V, g + C::G_W, tk);
                     fence_proxy_async_smem();
