@@ -26,7 +26,8 @@ every arrival of a completion to every wait for it.  Three properties are checke
   for the next one while the skipped one is still open would see the open phase's
   parity as done.
 
-`chunkwise_protocol(...)` writes the kernel's protocol.  Two earlier forms, which
+`chunkwise_protocol(...)` writes the chunkwise kernel's protocol and
+`summary_protocol(...)` that of the segment summary kernel (csrc/segments.cu).  Two earlier forms, which
 the overrun check rejects: `paired=False`, one B_OPS barrier and one B_VT barrier
 for two V stages; `exact_v_wait=True`, the token group waiting for an exact chunk's
 V with one V stage.
@@ -35,7 +36,7 @@ from __future__ import annotations
 
 from collections import defaultdict, deque
 
-COUNT = {"K_EMPTY": 2, "Q_EMPTY": 2, "G_EMPTY": 3, "CONV_SPLIT": 2}
+COUNT = {"K_EMPTY": 2, "Q_EMPTY": 2, "G_EMPTY": 3, "CONV_SPLIT": 2, "KV_EMPTY": 2}
 
 
 def _base(name: str) -> str:
@@ -273,4 +274,39 @@ def chunkwise_protocol(nc: int, vst: int, big: bool, exact=(), ng: int = 4, pair
             P.wait("token", s2("V_FULL", j), j)
             if paired or not ex[j]:
                 P.arrive("token", vt2(j), vt_tag(j))
+    return P
+
+
+def summary_protocol(nc: int, stages: int, ring: int = 4) -> Protocol:
+    """The hand-offs of the segment summary kernel (csrc/segments.cu) for nc chunks:
+    `stages` k/v stages (the first `stages` copies issued before the gate scan), a
+    weight ring of `ring` slots filled by two warps (even and odd chunks)."""
+    P = Protocol()
+    st = lambda name, c: f"{name}{c % stages}"
+    wr = lambda name, c: f"{name}{c % ring}"
+    # TMA producer
+    for c in range(min(stages, nc)):
+        P.arrive("tma", st("KV_FULL", c), c)
+    for c in range(stages, nc):
+        P.wait("tma", st("KV_EMPTY", c), c - stages)
+        P.arrive("tma", st("KV_FULL", c), c)
+    # MMA issuer
+    for c in range(nc):
+        P.wait("mma", st("VS", c), c)
+        P.arrive("mma", st("KV_EMPTY", c), c)
+    P.arrive("mma", "DONE", 0)
+    # weight warps
+    for w in (0, 1):
+        for c in range(w, nc, 2):
+            if c >= ring:
+                P.wait(f"weights{w}", wr("W_EMPTY", c), c - ring)
+            P.arrive(f"weights{w}", wr("W_FULL", c), c)
+    # compute group: w V in place, then n_seg from k
+    for c in range(nc):
+        P.wait("compute", st("KV_FULL", c), c)
+        P.wait("compute", wr("W_FULL", c), c)
+        P.arrive("compute", st("VS", c), c)
+        P.arrive("compute", wr("W_EMPTY", c), c)
+        P.arrive("compute", st("KV_EMPTY", c), c)
+    P.wait("compute", "DONE", 0)
     return P

@@ -8,7 +8,7 @@ import itertools
 
 import pytest
 
-from barrier_protocol import chunkwise_protocol
+from barrier_protocol import chunkwise_protocol, summary_protocol
 
 PATTERNS = [(), (0,), (1,), (0, 1), (2, 3, 5), (1, 3, 5, 7), tuple(range(9))]
 
@@ -54,3 +54,10 @@ def test_checker_finds_an_underrun():
     P = chunkwise_protocol(4, 1, False, (1,))
     P.roles["token"] = [op for op in P.roles["token"] if op[1] not in ("S_FULL", "UPD_DONE", "H_FULL")]
     assert any(p.startswith("underrun: the wait of token for V_FULL") for p in P.check())
+
+
+@pytest.mark.parametrize("stages", [4, 6, 8])
+@pytest.mark.parametrize("nc", [1, 3, 5, 8, 13, 40])
+def test_summary_protocol_has_no_deadlock_or_overrun(stages, nc):
+    problems = summary_protocol(nc, stages).check()
+    assert not problems, (stages, nc, problems[:3])
