@@ -16,7 +16,9 @@ xlstm_mlstm_step call per step and counts B tokens per step.
 value      tokens/s (B*T positions per step) with inputs resident in HBM,
            timed with CUDA events on the launch stream, max over ranks;
 e2e        the same call fed from pinned host buffers, H2D of the inputs and
-           D2H of h~ and the final state inside the timed region;
+           D2H of h~ and the final state inside the timed region, every step;
+           two steps in flight (copy-in, call and copy-out on three streams,
+           two sets of device buffers), as a serving loop runs it;
 roofline   algorithmic bytes per launch / launch time against the measured
            HBM copy bandwidth (the kernel is HBM-bound: 136 flop/B < ridge);
 cpu_baseline  the float64 oracle on a bounded sample of the same workload.
@@ -328,6 +330,12 @@ def _gate_overlap_split(w, dev):
     return first >= per_seq and idle >= 1 and first <= 4 * idle
 
 
+def capi_output_stage(o):
+    """The bf16-o~, bf16-h output stage descriptor for device tensor o."""
+    from xlstm_mlstm_matrix_b200 import capi
+    return capi.xlstm_mlstm_output_t(o.data_ptr(), capi.XLSTM_BF16, capi.XLSTM_BF16)
+
+
 class _Sequence:
     """One chunkwise forward over the whole batch per step (gated: through the
     output stage, bf16 o~ in and bf16 h out)."""
@@ -389,18 +397,43 @@ class _Sequence:
 
     def check_status(self):
         from xlstm_mlstm_matrix_b200 import capi
-        st, where = capi.xlstm_mlstm_workspace_status(self.ws, self.stream)
-        if st != 0:
-            raise capi.XlstmError(st, f"device status (where={where})")
+        for ws in [self.ws] + getattr(self, "e2e_ws", []):
+            st, where = capi.xlstm_mlstm_workspace_status(ws, self.stream)
+            if st != 0:
+                raise capi.XlstmError(st, f"device status (where={where})")
 
-    def host_buffers(self):
-        """Pinned host copies of the step's inputs and result buffers."""
+    def e2e_slots(self, n=2):
+        """n sets of device buffers for the end-to-end leg, each with pinned host
+        copies of the step's inputs and result buffers and a call on its own device
+        buffers: [(pairs_in [(dev, host)], pairs_out [(host, dev)], run)]."""
+        import ctypes
         import torch
         hin = [None if t is None else t.cpu().pin_memory() for t in self.ins]
-        hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in self.outs]
-        pairs_in = [(d, s) for d, s in zip(self.ins, hin) if d is not None]
-        pairs_out = list(zip(hout, self.outs))
-        return pairs_in, pairs_out
+        P = lambda t: None if t is None else ctypes.c_void_p(t.data_ptr())
+        slots = []
+        for k in range(n):
+            ins = self.ins if k == 0 else [None if t is None else torch.empty_like(t) for t in self.ins]
+            outs = self.outs if k == 0 else [torch.empty_like(t) for t in self.outs]
+            ws = self.ws if k == 0 else torch.zeros_like(self.ws)
+            if k > 0:
+                self.e2e_ws = getattr(self, "e2e_ws", []) + [ws]
+            if self.gated:
+                ost = capi_output_stage(ins[-1])
+                argv = (self.argv[0], ctypes.byref(ost), *(P(t) for t in ins[:-1]), *(P(t) for t in outs), P(ws),
+                        ws.numel(), ctypes.c_void_p(self.stream.cuda_stream))
+            else:
+                ost = None
+                argv = (self.argv[0], *(P(t) for t in ins), *(P(t) for t in outs), P(ws), ws.numel(),
+                        ctypes.c_void_p(self.stream.cuda_stream))
+
+            def run(argv=argv, ost=ost):
+                st = self.fn(*argv)
+                if st != 0:
+                    from xlstm_mlstm_matrix_b200 import capi
+                    raise capi.XlstmError(st, self.name)
+            hout = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in outs]
+            slots.append(([(d, h) for d, h in zip(ins, hin) if d is not None], list(zip(hout, outs)), run))
+        return slots
 
 
 class _Decode:
@@ -447,18 +480,30 @@ class _Decode:
     def check_status(self):
         pass
 
-    def host_buffers(self):
-        """Pinned host copies of one step's inputs (q, k, v, gates) and of h~;
-        the state stays resident on the device, as in a decode loop."""
+    def e2e_slots(self, n=2):
+        """n sets of device buffers for one step's inputs (q, k, v, gates) and h~,
+        with pinned host copies; the state stays resident on the device and every
+        step updates it in place, in order on the launch stream, as in a decode loop."""
+        import ctypes
         import torch
         j = 0
         hin = [self.q[j].cpu().pin_memory(), self.k[j].cpu().pin_memory(),
                self.v[j].cpu().pin_memory(), self.ig[j].cpu().pin_memory(),
                self.fg[j].cpu().pin_memory()]
-        self.dev_in = [torch.empty_like(t, device=self.h.device) for t in hin]
-        pairs_in = list(zip(self.dev_in, hin))
-        pairs_out = [(torch.empty(self.h.shape, dtype=self.h.dtype).pin_memory(), self.h)]
-        return pairs_in, pairs_out
+        slots = []
+        for k in range(n):
+            dev_in = [torch.empty_like(t, device=self.h.device) for t in hin]
+            h = self.h if k == 0 else torch.empty_like(self.h)
+
+            def run(dev_in=dev_in, h=h):
+                P = self.P
+                st = self.fn(ctypes.byref(self.desc), *(P(t) for t in dev_in), P(self.C), P(self.n), P(self.m),
+                             P(h), P(self.C), P(self.n), P(self.m), self.cs)
+                if st != 0:
+                    from xlstm_mlstm_matrix_b200 import capi
+                    raise capi.XlstmError(st, self.name)
+            slots.append((list(zip(dev_in, hin)), [(torch.empty(h.shape, dtype=h.dtype).pin_memory(), h)], run))
+        return slots
 
 
 class _Backward:
@@ -667,33 +712,52 @@ def run_ours(args, rank, world, local_rank):
     e2e_steps = 0 if args.no_e2e else max(1, min(args.steps, 5 if not w.steps else args.steps))
     e2e = None
     if e2e_steps:
-        pairs_in, pairs_out = job.host_buffers()
-        h2d = sum(s.numel() * s.element_size() for _, s in pairs_in)
-        d2h = sum(d.numel() * d.element_size() for d, _ in pairs_out)
+        # Two steps in flight: step i copies its inputs in on s_in, runs on the launch
+        # stream and copies its results out on s_out, with device buffer set i % 2; step
+        # i+2 reuses a set once step i's call has read its inputs and its results have
+        # been copied out.  Every step's copies are inside the timed region.
+        slots = job.e2e_slots(2)
+        h2d = sum(s.numel() * s.element_size() for _, s in slots[0][0])
+        d2h = sum(d.numel() * d.element_size() for d, _ in slots[0][1])
+        s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+        ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "call", "out")}
 
         def e2e_step(i):
-            for dst, src in pairs_in:
-                dst.copy_(src, non_blocking=True)
-            if w.steps:
-                job.step(i, src=[d for d, _ in pairs_in])
-            else:
-                job.step(i)
-            for dst, src in pairs_out:
-                dst.copy_(src, non_blocking=True)
+            k = i % 2
+            pairs_in, pairs_out, run = slots[k]
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev["call"][k])
+                for dst, src in pairs_in:
+                    dst.copy_(src, non_blocking=True)
+                ev["in"][k].record(s_in)
+            stream.wait_event(ev["in"][k])
+            if i >= 2:
+                stream.wait_event(ev["out"][k])
+            with torch.cuda.stream(stream):
+                run()
+                ev["call"][k].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev["call"][k])
+                for dst, src in pairs_out:
+                    dst.copy_(src, non_blocking=True)
+                ev["out"][k].record(s_out)
 
-        with torch.cuda.stream(stream):
-            e2e_step(0)
-            stream.synchronize()
-            barrier()
-            e0.record(stream)
-            for i in range(e2e_steps):
-                e2e_step(i)
-            e1.record(stream)
-            e1.synchronize()
+        for i in range(2):   # warm-up of both buffer sets
+            e2e_step(i)
+        torch.cuda.synchronize(dev)
+        barrier()
+        e0.record(s_in)
+        for i in range(e2e_steps):
+            e2e_step(i)
+        stream.wait_stream(s_out)
+        e1.record(stream)
+        e1.synchronize()
         barrier()
         e2e_ms = slowest(e0.elapsed_time(e1) / e2e_steps)
         e2e = {"value": job_rate(tokens, world, e2e_ms), "unit": UNIT,
-               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms}
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms,
+               "pipeline": "two steps in flight: H2D, call and D2H on three streams"}
         if w.steps:
             e2e["note"] = "per step: H2D of q, k, v and gates, D2H of h~; state resident on the device"
         job.check_status()
