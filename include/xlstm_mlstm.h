@@ -145,9 +145,16 @@ typedef struct {
  * B*H*T*d_v elements of h_dtype.  Invalid dtypes or a misaligned o_pre give
  * XLSTM_ERR_INVALID_ARG.  The state outputs are the recurrence's, untouched by
  * the gate.  On the tensor-core path the chunkwise kernel stores h~ in h_dtype
- * and a second, streaming kernel on the same stream applies the gate in place
- * (with a bf16 h, h~ is rounded to bf16 before the gate and the gated value
- * again); on the fp32 CUDA-core path the gate is applied in the epilogue.
+ * and a streaming kernel applies the gate in place (with a bf16 h, h~ is rounded
+ * to bf16 before the gate and the gated value again); on the fp32 CUDA-core path
+ * the gate is applied in the epilogue.  When the tensor-core grid ends in a
+ * partial wave, the call splits it in two launches on `stream`. It gates the
+ * first launch's h~ on a second stream of the library's own (one per device,
+ * made on the first such call and kept) while the second launch runs. The
+ * caller's stream waits for that gate before its last kernel, so all of the
+ * call's work is ordered on `stream` as usual, CUDA-graph capture included
+ * (the second stream joins the capture through events).  Make the first such
+ * call on a device outside a capture: it creates that stream and its events.
  */
 XLSTM_API xlstm_status_t xlstm_mlstm_fwd_chunkwise_out(
     const xlstm_mlstm_desc_t *desc, const xlstm_mlstm_output_t *out,
