@@ -61,3 +61,37 @@ def test_checker_finds_an_underrun():
 def test_summary_protocol_has_no_deadlock_or_overrun(stages, nc):
     problems = summary_protocol(nc, stages).check()
     assert not problems, (stages, nc, problems[:3])
+
+
+def _kernel_barriers(path, prefix):
+    import os
+    import re
+    root = os.path.join(os.path.dirname(__file__), "..", "xlstm_mlstm_matrix_b200", "csrc")
+    src = open(os.path.join(root, path)).read()
+    return set(re.findall(r"bar\[" + re.escape(prefix) + r"(B_[A-Z0-9_]+)", src))
+
+
+def _model_barriers(P):
+    import re
+    # model names: kernel names without "B_", slot digits appended; CONV_SPLIT / CONV_CLO
+    # stand for B_CONV0 / B_CONV1
+    names = {re.sub(r"\d+$", "", bar) for ops in P.roles.values() for _, bar, _ in ops}
+    names = {"CONV" if n.startswith("CONV_") else n for n in names}
+    return {"B_" + n for n in names}
+
+
+def test_model_covers_every_barrier_of_the_chunkwise_kernel():
+    """The model names every hand-off barrier the kernel waits on or arrives at (the
+    drain barrier, used by one thread alone at teardown, aside); a barrier added to
+    the kernel without the model fails here."""
+    used = _kernel_barriers("chunkwise_tc.cu", "") - {"B_DRAIN"}
+    used = {"B_CONV" if n.startswith("B_CONV") else n for n in used}
+    modelled = set()
+    for vst, big in ((2, False), (2, True), (1, False)):
+        modelled |= _model_barriers(chunkwise_protocol(4, vst, big, (1,)))
+    assert used == modelled, (used - modelled, modelled - used)
+
+
+def test_model_covers_every_barrier_of_the_summary_kernel():
+    used = _kernel_barriers("segments.cu", "C::") - {"B_DRAIN"}
+    assert used == _model_barriers(summary_protocol(6, 4)), used
